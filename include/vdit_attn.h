@@ -1,0 +1,139 @@
+/*
+ * vdit_attn.h -- C ABI of the bf16 video-DiT attention forward library
+ * (libvdit_attn.so, sm_100a / B200).
+ *
+ * The operation is the forward multi-head attention over the flattened
+ * spatiotemporal latent tokens of a video diffusion transformer:
+ *
+ *   O[b,i,h,:] = sum_{j in A(i)} softmax_j(scale * q[b,i,h,:] . k[b,j,h,:]) v[b,j,h,:]
+ *   LSE[b,h,i] = ln sum_{j in A(i)} exp(scale * q[b,i,h,:] . k[b,j,h,:])
+ *
+ * Sources for the operation:
+ *  - "VC-Attention" (aikraft.ru), section 01 "Why attention became the
+ *    bottleneck": the clip is flattened into one sequence of spatiotemporal
+ *    tokens and full self-attention runs in every transformer layer; on B200
+ *    the FP32 exp + cast between the two matrix products is the longest
+ *    stage.
+ *  - "Realtime video generation: FLOPS calculation and optimizations"
+ *    (sudonull.com), FLOP list: self-attention (~82% of the layer at
+ *    S = 75,600) and text->video cross-attention in each of the 40 layers;
+ *    the FlashAttention bullet: no 75K x 75K score matrix is materialised.
+ *  - Wave Forcing digest (airadar.tv), summary: block-causal attention in
+ *    which later chunks read the K/V of earlier chunks.
+ *
+ * Conventions shared by every entry point:
+ *  - Layout BSHD, contiguous: q and o are [B][Sq][H][D], k and v are
+ *    [B][Skv][H][D], all bf16 (IEEE binary16 "brain" format, raw 2-byte
+ *    elements).  lse is [B][H][Sq] fp32, natural log, unnormalised
+ *    (LSE = max + ln(sum exp(logit - max))).
+ *  - D must be 128.
+ *  - Pointers are DEVICE pointers on the current CUDA device, 16-byte
+ *    aligned, owned by the caller; the library never frees, keeps or
+ *    allocates device memory on behalf of a call.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls are asynchronous on that stream.
+ *  - Argument errors are detected on the host before any launch and return
+ *    a status with nothing launched.  No C++ exception crosses the ABI.
+ *  - The library keeps no mutable per-call host state; concurrent calls from
+ *    several host threads are safe.
+ */
+#ifndef VDIT_ATTN_H
+#define VDIT_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VDIT_ATTN_ABI_VERSION 1
+
+/* Mask kinds.  A(i) is the set of keys query row i may attend to. */
+typedef enum {
+    /* A(i) = all keys j < Skv.  Bidirectional self-attention. */
+    VDIT_MASK_FULL = 0,
+    /* A(i) = { j : floor(j / c) <= floor(i / c) }, c = chunk_tokens.
+     * Chunks are contiguous from token 0; the last may be partial.  Requires
+     * Sq == Skv.  Keys of later chunks are skipped, not just masked. */
+    VDIT_MASK_BLOCK_CAUSAL = 1,
+    /* Same arithmetic as FULL; the caller says the keys are a short text
+     * sequence (Skv << Sq), e.g. 512 text tokens. */
+    VDIT_MASK_CROSS = 2
+} vdit_mask_kind;
+
+typedef enum {
+    VDIT_OK = 0,
+    VDIT_ERR_INVALID_ARG = 1,  /* null pointer, negative size, Skv == 0,
+                                  bad mask_kind, chunk_tokens < 1 with
+                                  BLOCK_CAUSAL, Sq != Skv with BLOCK_CAUSAL,
+                                  scale not finite or <= 0, H or B > 65535 */
+    VDIT_ERR_UNSUPPORTED = 2,  /* D != 128, or the device is not sm_100 */
+    VDIT_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned */
+    VDIT_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
+    VDIT_ERR_TIMEOUT = 5,      /* a kernel gave up waiting on one of its own
+                                  pipeline barriers (reported by
+                                  vdit_get_device_status) */
+    VDIT_ERR_WORKSPACE = 6     /* workspace missing or too small */
+} vdit_status;
+
+/*
+ * vdit_attn_plan -- host-only query, touches no device.
+ * Writes the workspace size the _ws entry point needs (0 for every shape in
+ * this version) and, if grid_ctas is non-NULL, the number of CTAs the
+ * forward launches.  Same argument rules as vdit_attn_fwd, except that
+ * pointers are not involved.
+ */
+vdit_status vdit_attn_plan(int B, int H, int Sq, int Skv, int D, int mask_kind,
+                           int chunk_tokens, size_t* workspace_bytes,
+                           int* grid_ctas);
+
+/*
+ * vdit_attn_fwd -- launch the attention forward on `stream`.
+ *   q, k, v : device bf16 inputs (see conventions above).
+ *   o       : device bf16 output, [B][Sq][H][D]; must not alias q/k/v.
+ *   lse     : device fp32 output [B][H][Sq], or NULL to skip it.
+ *   scale   : multiplies q.k before the softmax (1/sqrt(D) for the Wan
+ *             configurations); finite and > 0.
+ *   mask_kind, chunk_tokens : see vdit_mask_kind; chunk_tokens is ignored
+ *             unless mask_kind == VDIT_MASK_BLOCK_CAUSAL.
+ * B == 0, H == 0 or Sq == 0 is a valid empty call: VDIT_OK, nothing launched.
+ * Returns VDIT_ERR_CUDA if the launch itself fails.  Timeouts inside the
+ * kernel are reported later by vdit_get_device_status.
+ */
+vdit_status vdit_attn_fwd(const void* q, const void* k, const void* v, void* o,
+                          float* lse, int B, int H, int Sq, int Skv, int D,
+                          float scale, int mask_kind, int chunk_tokens,
+                          void* stream);
+
+/*
+ * vdit_attn_fwd_ws -- vdit_attn_fwd with a caller-owned device workspace of
+ * `workspace_bytes` bytes (at least what vdit_attn_plan reports; NULL is
+ * accepted when that is 0).
+ */
+vdit_status vdit_attn_fwd_ws(const void* q, const void* k, const void* v,
+                             void* o, float* lse, int B, int H, int Sq,
+                             int Skv, int D, float scale, int mask_kind,
+                             int chunk_tokens, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/*
+ * vdit_get_device_status -- synchronises `stream`, then reads and clears the
+ * current device's error word that the kernels set when a bounded wait on
+ * one of their pipeline barriers runs out.  Returns VDIT_OK,
+ * VDIT_ERR_TIMEOUT, or VDIT_ERR_CUDA if the synchronisation itself failed.
+ * If `detail` is non-NULL it receives the raw error word (0 when clean).
+ */
+vdit_status vdit_get_device_status(void* stream, uint32_t* detail);
+
+/* Static, human-readable name of a status code. */
+const char* vdit_status_string(int status);
+
+/* VDIT_ATTN_ABI_VERSION of the loaded library. */
+int vdit_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VDIT_ATTN_H */

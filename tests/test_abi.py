@@ -1,0 +1,95 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+declared in include/vdit_attn.h, and rejects bad arguments on the host before
+touching the device."""
+import os
+import re
+
+import pytest
+
+from video_diffusion_transformer_attention_b200 import binding as vb
+from video_diffusion_transformer_attention_b200.build import build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "vdit_attn.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_library():
+    build()
+    return vb.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vdit_\w+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert declared_functions() == sorted(vb.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    h = vb.lib()
+    for name in declared_functions():
+        assert hasattr(h, name), name
+
+
+def test_abi_version_and_status_strings():
+    assert vb.vdit_abi_version() == 1
+    assert vb.vdit_status_string(vb.VDIT_OK) == "VDIT_OK"
+    assert vb.vdit_status_string(vb.VDIT_ERR_TIMEOUT) == "VDIT_ERR_TIMEOUT"
+    assert vb.vdit_status_string(999) == "VDIT_ERR_UNKNOWN"
+
+
+def test_plan_reports_grid_and_zero_workspace():
+    ws, grid = vb.vdit_attn_plan(1, 40, 75600, 75600, 128, vb.VDIT_MASK_FULL, 0)
+    assert ws == 0 and grid == 296 * 40
+    ws, grid = vb.vdit_attn_plan(2, 3, 300, 300, 128, vb.VDIT_MASK_BLOCK_CAUSAL, 100)
+    assert grid == 2 * 3 * 2
+    assert vb.vdit_attn_plan(1, 1, 0, 5, 128, 0, 0) == (0, 0)
+
+
+@pytest.mark.parametrize("args,status", [
+    ((1, 1, 16, 16, 64, 0, 0), vb.VDIT_ERR_UNSUPPORTED),
+    ((1, 1, 16, 0, 128, 0, 0), vb.VDIT_ERR_INVALID_ARG),
+    ((1, 1, 16, 16, 128, 3, 0), vb.VDIT_ERR_INVALID_ARG),
+    ((1, 1, 16, 16, 128, 1, 0), vb.VDIT_ERR_INVALID_ARG),
+    ((1, 1, 16, 32, 128, 1, 8), vb.VDIT_ERR_INVALID_ARG),
+    ((-1, 1, 16, 16, 128, 0, 0), vb.VDIT_ERR_INVALID_ARG),
+    ((1, 70000, 16, 16, 128, 0, 0), vb.VDIT_ERR_INVALID_ARG),
+])
+def test_plan_rejects_bad_shapes(args, status):
+    with pytest.raises(vb.VditError) as e:
+        vb.vdit_attn_plan(*args)
+    assert e.value.status == status
+
+
+A = 1 << 20  # a fake, 16-byte aligned "device" address: never dereferenced
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), vb.VDIT_ERR_INVALID_ARG),
+    (dict(o=None), vb.VDIT_ERR_INVALID_ARG),
+    (dict(q=A + 2), vb.VDIT_ERR_MISALIGNED),
+    (dict(lse=A * 9 + 4), vb.VDIT_ERR_MISALIGNED),
+    (dict(scale=0.0), vb.VDIT_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), vb.VDIT_ERR_INVALID_ARG),
+    (dict(scale=-1.0), vb.VDIT_ERR_INVALID_ARG),
+    (dict(D=96), vb.VDIT_ERR_UNSUPPORTED),
+    (dict(o=A), vb.VDIT_ERR_INVALID_ARG),  # output aliases q
+    (dict(mask_kind=1, chunk_tokens=0), vb.VDIT_ERR_INVALID_ARG),
+])
+def test_fwd_rejects_bad_arguments_before_any_launch(kw, status):
+    args = dict(q=A, k=A * 3, v=A * 5, o=A * 7, lse=A * 9, B=1, H=2, Sq=64, Skv=64, D=128,
+                scale=0.1, mask_kind=0, chunk_tokens=0)
+    args.update(kw)
+    st = vb.vdit_attn_fwd(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"], args["H"],
+                          args["Sq"], args["Skv"], args["D"], args["scale"], args["mask_kind"],
+                          args["chunk_tokens"], stream=0, check=False)
+    assert st == status
+
+
+def test_empty_call_is_a_no_op():
+    for B, H, Sq in [(0, 2, 64), (1, 0, 64), (1, 2, 0)]:
+        assert vb.vdit_attn_fwd(None, None, None, None, None, B, H, Sq, 64, 128, 0.1, 0, 0,
+                                stream=0, check=False) == vb.VDIT_OK

@@ -1,0 +1,164 @@
+"""ctypes binding of libvdit_attn.so: the C ABI of include/vdit_attn.h, same names.
+
+Argument marshalling only -- every step of the attention runs in the CUDA
+library.  Functions accept raw integers (device addresses, a cudaStream_t
+value) or torch tensors / streams, which are turned into those integers.
+If the library has not been built, loading raises ``ImportError``; there is no
+fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libvdit_attn.so")
+
+VDIT_MASK_FULL = 0
+VDIT_MASK_BLOCK_CAUSAL = 1
+VDIT_MASK_CROSS = 2
+
+VDIT_OK = 0
+VDIT_ERR_INVALID_ARG = 1
+VDIT_ERR_UNSUPPORTED = 2
+VDIT_ERR_MISALIGNED = 3
+VDIT_ERR_CUDA = 4
+VDIT_ERR_TIMEOUT = 5
+VDIT_ERR_WORKSPACE = 6
+
+# every entry point of include/vdit_attn.h
+EXPORTS = (
+    "vdit_attn_plan",
+    "vdit_attn_fwd",
+    "vdit_attn_fwd_ws",
+    "vdit_get_device_status",
+    "vdit_status_string",
+    "vdit_abi_version",
+)
+
+_lock = threading.Lock()
+_lib = None
+
+
+class VditError(RuntimeError):
+    """A non-OK status returned by the library."""
+
+    def __init__(self, status: int, what: str):
+        self.status = int(status)
+        super().__init__(f"{what}: {vdit_status_string(status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """Load (once) and return the library handle."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(
+                    f"{LIB_PATH} is missing; build it with "
+                    "`python -m video_diffusion_transformer_attention_b200.build`")
+            h = ctypes.CDLL(LIB_PATH)
+            c_int, c_float, c_size, vp = ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p
+            h.vdit_attn_plan.restype = c_int
+            h.vdit_attn_plan.argtypes = [c_int] * 7 + [ctypes.POINTER(c_size), ctypes.POINTER(c_int)]
+            fwd_args = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_float, c_int, c_int]
+            h.vdit_attn_fwd.restype = c_int
+            h.vdit_attn_fwd.argtypes = fwd_args + [vp]
+            h.vdit_attn_fwd_ws.restype = c_int
+            h.vdit_attn_fwd_ws.argtypes = fwd_args + [vp, c_size, vp]
+            h.vdit_get_device_status.restype = c_int
+            h.vdit_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
+            h.vdit_status_string.restype = ctypes.c_char_p
+            h.vdit_status_string.argtypes = [c_int]
+            h.vdit_abi_version.restype = c_int
+            h.vdit_abi_version.argtypes = []
+            _lib = h
+    return _lib
+
+
+def _addr(x) -> int | None:
+    """A device address from a tensor, an int, or None."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return int(x.data_ptr())
+
+
+def _stream(s) -> int | None:
+    """A cudaStream_t value from a torch stream, an int, or None (current stream)."""
+    if s is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream) if torch.cuda.is_available() else None
+    if isinstance(s, int):
+        return s
+    return int(s.cuda_stream)
+
+
+def vdit_status_string(status: int) -> str:
+    return lib().vdit_status_string(int(status)).decode()
+
+
+def vdit_abi_version() -> int:
+    return int(lib().vdit_abi_version())
+
+
+def vdit_attn_plan(B, H, Sq, Skv, D, mask_kind, chunk_tokens):
+    """Returns (workspace_bytes, grid_ctas); raises VditError on a bad shape."""
+    ws = ctypes.c_size_t(0)
+    grid = ctypes.c_int(0)
+    st = lib().vdit_attn_plan(B, H, Sq, Skv, D, mask_kind, chunk_tokens, ctypes.byref(ws), ctypes.byref(grid))
+    if st != VDIT_OK:
+        raise VditError(st, "vdit_attn_plan")
+    return int(ws.value), int(grid.value)
+
+
+def vdit_attn_fwd(q, k, v, o, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, stream=None,
+                  check=True) -> int:
+    """Launch the forward; returns the status (raises VditError if check and not OK)."""
+    st = lib().vdit_attn_fwd(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), B, H, Sq, Skv, D,
+                             float(scale), mask_kind, chunk_tokens, _stream(stream))
+    if check and st != VDIT_OK:
+        raise VditError(st, "vdit_attn_fwd")
+    return st
+
+
+def vdit_attn_fwd_ws(q, k, v, o, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, workspace,
+                     workspace_bytes, stream=None, check=True) -> int:
+    st = lib().vdit_attn_fwd_ws(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), B, H, Sq, Skv, D,
+                                float(scale), mask_kind, chunk_tokens, _addr(workspace),
+                                int(workspace_bytes), _stream(stream))
+    if check and st != VDIT_OK:
+        raise VditError(st, "vdit_attn_fwd_ws")
+    return st
+
+
+def vdit_get_device_status(stream=None):
+    """Returns (status, raw error word); synchronises the stream."""
+    word = ctypes.c_uint32(0)
+    st = lib().vdit_get_device_status(_stream(stream), ctypes.byref(word))
+    return int(st), int(word.value)
+
+
+def attention(q, k, v, scale=None, mask_kind=VDIT_MASK_FULL, chunk_tokens=0, out=None, lse=None,
+              return_lse=True, stream=None):
+    """Convenience wrapper over vdit_attn_fwd for CUDA bf16 tensors in [B, S, H, D].
+
+    Output buffers are allocated with torch when not given (torch only serves
+    as the device-memory allocator here).  Returns (o, lse) or o.
+    """
+    import torch
+    B, Sq, H, D = q.shape
+    Skv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / float(D) ** 0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    for t in (q, k, v, out):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError("q, k, v, out must be contiguous CUDA bf16 tensors")
+    vdit_attn_fwd(q, k, v, out, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, stream)
+    return (out, lse) if return_lse else out

@@ -1,0 +1,444 @@
+// attn_fwd_sm100.cuh -- warp-specialised bf16 attention forward for sm_100a.
+//
+// One CTA owns two 128-row query tiles of one (batch, head) and streams the
+// key/value sequence through shared memory in 128-key tiles:
+//
+//   S_t = Q_t K_j^T               tcgen05.mma, both operands in smem, fp32 acc in TMEM
+//   P_t = exp2(S_t*scale*log2e - m_t)   softmax warps, registers, P back to TMEM as bf16
+//   O_t += P_t V_j                tcgen05.mma, P from TMEM, V from smem
+//
+// This is the streaming ("online") softmax that avoids materialising the
+// S x S score matrix -- the FlashAttention bullet of "Realtime video
+// generation: FLOPS calculation and optimizations" (sudonull.com) -- with
+// the running row maximum and row sum kept per query row ("VC-Attention"
+// (aikraft.ru), section 02, Restore step: the online softmax already holds
+// the row sum).  The exp + cast between the two products is the long pole on
+// B200 (same page, section 01), so the softmax runs in two warpgroups that
+// alternate with the tensor core: while warpgroup 0 exponentiates tile 0,
+// the tensor core computes P_1 V and S_1 for tile 1, and vice versa.
+//
+// Roles (320 threads):
+//   warps 0-3  softmax + correction + epilogue of query tile 0
+//   warps 4-7  softmax + correction + epilogue of query tile 1
+//   warp  8    TMA producer (Q once, then K_j, V_j into a 4-slot ring)
+//   warp  9    TMEM allocator and single-thread tcgen05.mma issuer
+//
+// TMEM (512 columns x 128 lanes, fp32): S_0 [0,128), S_1 [128,256),
+// O_0 [256,384), O_1 [384,512).  P_t (bf16, two per column) overwrites the
+// first 64 columns of S_t; query row r of a tile lives in TMEM lane r.
+//
+// Every wait on a pipeline barrier is bounded: when it runs out the CTA
+// raises a shared abort flag, ORs a code into the device status word, and
+// every role leaves its loop so the CTA still reaches teardown.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace vdit {
+
+constexpr int kBlockM = 128;   // query rows per tile
+constexpr int kBlockN = 128;   // keys per K/V tile
+constexpr int kHeadDim = 128;  // D
+constexpr int kQTiles = 2;     // query tiles per CTA
+constexpr int kStages = 4;     // K/V ring slots (each holds one K or one V tile)
+constexpr int kTileBytes = kBlockM * kHeadDim * 2;  // 32 KB
+constexpr int kHalfBytes = kTileBytes / 2;          // 128 rows x 64 bf16, 128B-swizzled
+constexpr int kNumThreads = 320;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
+
+constexpr int kMaskFull = 0;
+constexpr int kMaskBlockCausal = 1;
+constexpr int kMaskCross = 2;
+
+// Device status word codes (OR-ed together).
+constexpr uint32_t kStatusTimeout = 1u;
+constexpr uint32_t kSiteProducer = 1u << 8;
+constexpr uint32_t kSiteMma = 1u << 9;
+constexpr uint32_t kSiteSoftmax = 1u << 10;
+
+struct __align__(8) Barriers {
+    uint64_t q_full[kQTiles];
+    uint64_t kv_full[kStages];
+    uint64_t kv_empty[kStages];
+    uint64_t s_full[kQTiles];
+    uint64_t p_full[kQTiles];
+    uint64_t o_full[kQTiles];
+    uint64_t drain;  // MMA issuer's own completion barrier on the abort path
+    uint32_t tmem_base;
+    int abort;
+};
+
+constexpr int kSmemQ = 0;
+constexpr int kSmemKV = kQTiles * kTileBytes;
+constexpr int kSmemBar = kSmemKV + kStages * kTileBytes;
+constexpr int kSmemBytes = kSmemBar + int(sizeof(Barriers)) + 1024;  // + alignment slack
+
+struct FwdParams {
+    int B, H, Sq, Skv;
+    int mask_kind;
+    int chunk;
+    float scale_log2;  // scale * log2(e)
+    __nv_bfloat16* o;
+    float* lse;
+    unsigned long long timeout_ns;
+};
+
+// Written by kernels when a bounded wait runs out; read and cleared by the host.
+__device__ uint32_t g_status_word = 0;
+
+// ---------------------------------------------------------------- descriptors
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 format:
+// start address >> 4 in bits [0,14), leading byte offset >> 4 in [16,30),
+// stride byte offset >> 4 in [32,46), version 1 in [46,48), layout 2
+// (SWIZZLE_128B) in [61,64).
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return uint64_t((saddr & 0x3FFFFu) >> 4) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
+           (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator (bits [4,6) = 1),
+// A = B = bf16 ([7,10) = [10,13) = 1), A K-major, B K-major or MN-major
+// (bit 16), N >> 3 in [17,23), M >> 4 in [24,29).
+__host__ __device__ constexpr uint32_t make_idesc_bf16(bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+           (uint32_t(kBlockN >> 3) << 17) | (uint32_t(kBlockM >> 4) << 24);
+}
+
+// ---------------------------------------------------------------- waits
+
+__device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                             unsigned long long timeout_ns, uint32_t site) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0) {
+            if (*abort) return false;
+            if (global_timer_ns() - t0 > timeout_ns) {
+                *abort = 1;
+                atomicOr(&g_status_word, kStatusTimeout | site);
+                return false;
+            }
+        }
+    }
+}
+
+// All 32 lanes wait; the warp proceeds only if every lane saw the phase.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          unsigned long long timeout_ns, uint32_t site) {
+    const bool ok = bounded_wait(bar, parity, abort, timeout_ns, site);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// ---------------------------------------------------------------- MMA helpers
+
+// S[128 x 128] = Q_tile[128 x 128] * K_tile[128 x 128]^T, both K-major with
+// 128B swizzle, each stored as two 16 KB halves (head dims 0-63 and 64-127).
+// K = 16 per instruction: 4 steps of 32 bytes inside a half, then the next half.
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+    constexpr uint32_t idesc = make_idesc_bf16(false);
+#pragma unroll
+    for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+        const uint32_t off = uint32_t(kk >> 2) * kHalfBytes + uint32_t(kk & 3) * 32u;
+        umma_ss(d_tmem, smem_desc_sw128(q_smem + off, 16, 1024), smem_desc_sw128(k_smem + off, 16, 1024),
+                idesc, kk > 0 ? 1u : 0u);
+    }
+}
+
+// O[128 x 128] (+)= P[128 x 128 keys] * V_tile[128 keys x 128].  P comes from
+// TMEM (two bf16 per column, 8 columns per K = 16 step).  V is the B operand
+// in MN-major form: head dim is contiguous; 64-dim halves are 16 KB apart
+// (leading byte offset), 8-key row groups 1 KB apart (stride byte offset),
+// and each 16-key step advances 16 rows = 2 KB.
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem,
+                                         bool accumulate) {
+    constexpr uint32_t idesc = make_idesc_bf16(true);
+#pragma unroll
+    for (int kk = 0; kk < kBlockN / 16; ++kk) {
+        umma_ts(d_tmem, p_tmem + uint32_t(kk) * 8u, smem_desc_sw128(v_smem + uint32_t(kk) * 2048u, kHalfBytes, 1024),
+                idesc, (accumulate || kk > 0) ? 1u : 0u);
+    }
+}
+
+// ---------------------------------------------------------------- kernel
+
+__global__ void __launch_bounds__(kNumThreads, 1)
+    attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + (((raw_base + 1023u) & ~1023u) - raw_base);
+    Barriers* bars = reinterpret_cast<Barriers*>(smem + kSmemBar);
+    volatile int* abort_flag = &bars->abort;
+
+    const int warp = int(threadIdx.x >> 5);
+    const int lane = int(threadIdx.x & 31);
+    const int h = int(blockIdx.y);
+    const int b = int(blockIdx.z);
+    const int q0 = int(blockIdx.x) * (kQTiles * kBlockM);
+
+    if (threadIdx.x == 0) {
+        for (int t = 0; t < kQTiles; ++t) {
+            mbar_init(smem_addr(&bars->q_full[t]), 1);
+            mbar_init(smem_addr(&bars->s_full[t]), 1);
+            mbar_init(smem_addr(&bars->p_full[t]), 4 * 32);
+            mbar_init(smem_addr(&bars->o_full[t]), 1);
+        }
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(smem_addr(&bars->kv_full[s]), 1);
+            mbar_init(smem_addr(&bars->kv_empty[s]), 1);
+        }
+        mbar_init(smem_addr(&bars->drain), 1);
+        bars->abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == kLoadWarp && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(smem_addr(&bars->tmem_base), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = bars->tmem_base;
+
+    // Keys this CTA needs: all of them, or for block-causal everything up to
+    // the end of the chunk that holds the CTA's last valid query row.
+    int kv_end = p.Skv;
+    if (p.mask_kind == kMaskBlockCausal) {
+        const int last_row = min(q0 + kQTiles * kBlockM - 1, p.Sq - 1);
+        const long long lim = (static_cast<long long>(last_row / p.chunk) + 1) * p.chunk;
+        kv_end = static_cast<int>(min(static_cast<long long>(p.Skv), lim));
+    }
+    const int n_kv = (kv_end + kBlockN - 1) / kBlockN;
+
+    const uint32_t sQ = smem_addr(smem + kSmemQ);
+    const uint32_t sKV = smem_addr(smem + kSmemKV);
+
+    if (warp == kLoadWarp) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            for (int t = 0; t < kQTiles; ++t) {
+                const uint32_t bar = smem_addr(&bars->q_full[t]);
+                mbar_arrive_expect_tx(bar, kTileBytes);
+                tma_load_4d(sQ + t * kTileBytes, &tm_q, bar, 0, h, q0 + t * kBlockM, b);
+                tma_load_4d(sQ + t * kTileBytes + kHalfBytes, &tm_q, bar, 64, h, q0 + t * kBlockM, b);
+            }
+            for (int u = 0; u < 2 * n_kv; ++u) {
+                const int slot = u % kStages;
+                const uint32_t phase = uint32_t(u / kStages) & 1u;
+                if (!bounded_wait(smem_addr(&bars->kv_empty[slot]), phase ^ 1u, abort_flag, p.timeout_ns,
+                                  kSiteProducer))
+                    break;
+                const uint32_t full = smem_addr(&bars->kv_full[slot]);
+                const CUtensorMap* map = (u & 1) ? &tm_v : &tm_k;
+                const int row = (u >> 1) * kBlockN;
+                mbar_arrive_expect_tx(full, kTileBytes);
+                tma_load_4d(sKV + slot * kTileBytes, map, full, 0, h, row, b);
+                tma_load_4d(sKV + slot * kTileBytes + kHalfBytes, map, full, 64, h, row, b);
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
+            bool ok = bounded_wait(smem_addr(&bars->q_full[0]), 0, abort_flag, p.timeout_ns, kSiteMma) &&
+                      bounded_wait(smem_addr(&bars->q_full[1]), 0, abort_flag, p.timeout_ns, kSiteMma);
+            // prologue: S_0 and S_1 against K_0
+            int k_slot = 0;
+            if (ok) ok = bounded_wait(smem_addr(&bars->kv_full[0]), 0, abort_flag, p.timeout_ns, kSiteMma);
+            if (ok) {
+                tc_fence_after_sync();
+                issue_qk(tS0, sQ, sKV);
+                umma_commit(smem_addr(&bars->s_full[0]));
+                issue_qk(tS1, sQ + kTileBytes, sKV);
+                umma_commit(smem_addr(&bars->s_full[1]));
+                umma_commit(smem_addr(&bars->kv_empty[0]));
+            }
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int uv = 2 * j + 1;
+                const int v_slot = uv % kStages;
+                ok = bounded_wait(smem_addr(&bars->kv_full[v_slot]), uint32_t(uv / kStages) & 1u, abort_flag,
+                                  p.timeout_ns, kSiteMma) &&
+                     bounded_wait(smem_addr(&bars->p_full[0]), uint32_t(j) & 1u, abort_flag, p.timeout_ns,
+                                  kSiteMma);
+                if (!ok) break;
+                tc_fence_after_sync();
+                issue_pv(tO0, tS0, sKV + v_slot * kTileBytes, j > 0);
+                const bool more = (j + 1) < n_kv;
+                if (more) {
+                    const int uk = 2 * (j + 1);
+                    k_slot = uk % kStages;
+                    ok = bounded_wait(smem_addr(&bars->kv_full[k_slot]), uint32_t(uk / kStages) & 1u,
+                                      abort_flag, p.timeout_ns, kSiteMma);
+                    if (!ok) break;
+                    tc_fence_after_sync();
+                    issue_qk(tS0, sQ, sKV + k_slot * kTileBytes);
+                    umma_commit(smem_addr(&bars->s_full[0]));
+                } else {
+                    umma_commit(smem_addr(&bars->o_full[0]));
+                }
+                ok = bounded_wait(smem_addr(&bars->p_full[1]), uint32_t(j) & 1u, abort_flag, p.timeout_ns,
+                                  kSiteMma);
+                if (!ok) break;
+                tc_fence_after_sync();
+                issue_pv(tO1, tS1, sKV + v_slot * kTileBytes, j > 0);
+                umma_commit(smem_addr(&bars->kv_empty[v_slot]));
+                if (more) {
+                    issue_qk(tS1, sQ + kTileBytes, sKV + k_slot * kTileBytes);
+                    umma_commit(smem_addr(&bars->s_full[1]));
+                    umma_commit(smem_addr(&bars->kv_empty[k_slot]));
+                } else {
+                    umma_commit(smem_addr(&bars->o_full[1]));
+                }
+            }
+            if (!ok) {
+                // Let every MMA already issued finish before TMEM is released;
+                // this wait ignores the abort flag but keeps its time limit.
+                umma_commit(smem_addr(&bars->drain));
+                const uint32_t drain = smem_addr(&bars->drain);
+                const uint64_t t0 = global_timer_ns();
+                while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < p.timeout_ns) {
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------ softmax warpgroups
+        const int t = warp >> 2;        // query tile
+        const int quarter = warp & 3;   // TMEM lane quarter this warp may access
+        const int row_in_tile = quarter * 32 + lane;
+        const int row = q0 + t * kBlockM + row_in_tile;
+        const uint32_t lane_bits = uint32_t(quarter * 32) << 16;
+        const uint32_t tS = tmem + lane_bits + uint32_t(t) * 128u;
+        const uint32_t tO = tmem + lane_bits + 256u + uint32_t(t) * 128u;
+        const uint32_t s_full = smem_addr(&bars->s_full[t]);
+        const uint32_t p_full = smem_addr(&bars->p_full[t]);
+
+        int kv_lim = p.Skv;  // keys [0, kv_lim) are allowed for this row
+        if (p.mask_kind == kMaskBlockCausal) {
+            const long long lim = (static_cast<long long>(row / p.chunk) + 1) * p.chunk;
+            kv_lim = static_cast<int>(min(static_cast<long long>(p.Skv), lim));
+        }
+        const float scale_log2 = p.scale_log2;
+        float m = -INFINITY;  // reference max (log2 units) the exponentials are taken against
+        float l = 0.0f;       // running row sum at that reference
+        bool ok = true;
+
+        for (int j = 0; j < n_kv; ++j) {
+            ok = warp_wait(s_full, uint32_t(j) & 1u, abort_flag, p.timeout_ns, kSiteSoftmax);
+            if (!ok) break;
+            tc_fence_after_sync();
+            uint32_t s[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tS + uint32_t(c) * 32u, s[c]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld_wait(s[c]);
+
+            const int lim = kv_lim - j * kBlockN;
+            if (lim < kBlockN) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (c * 32 + i >= lim) s[c][i] = __float_as_uint(-INFINITY);
+            }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(s[c][i]));
+            const float m_tile = mx * scale_log2;
+
+            float alpha = 1.0f;
+            bool rescale = false;
+            if (j == 0) {
+                m = m_tile;
+            } else if (m_tile > m + kRescaleThreshold) {
+                alpha = ex2_approx(m - m_tile);
+                m = m_tile;
+                l *= alpha;
+                rescale = true;
+            }
+            const float m_use = (m == -INFINITY) ? 0.0f : m;
+            // P = exp2(S * scale*log2e - m) with the row sum in fp32; each pair
+            // is packed to bf16x2 into the register slot it has just consumed,
+            // and 16 packed columns at a time go back over S in TMEM.
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    const float p0 = ex2_approx(fmaf(__uint_as_float(s[c][i]), scale_log2, -m_use));
+                    const float p1 = ex2_approx(fmaf(__uint_as_float(s[c][i + 1]), scale_log2, -m_use));
+                    l += p0 + p1;
+                    s[c][i / 2] = pack_bf16x2(p0, p1);
+                }
+                tmem_st16(tS + uint32_t(c) * 16u, s[c]);
+            }
+            if (__any_sync(0xffffffffu, rescale)) {
+                // O_t holds sum_k P_k V_k at the old reference: bring it to the new one.
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + uint32_t(c) * 32u, o);
+                    tmem_ld_wait(o);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st32(tO + uint32_t(c) * 32u, o);
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before_sync();
+            mbar_arrive(p_full);
+        }
+
+        if (ok) ok = warp_wait(smem_addr(&bars->o_full[t]), 0, abort_flag, p.timeout_ns, kSiteSoftmax);
+        if (ok) {
+            tc_fence_after_sync();
+            const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
+            __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.Sq + row) * p.H + h) * kHeadDim;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tO + uint32_t(c) * 32u, o);
+                tmem_ld_wait(o);
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+                if (row < p.Sq) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                }
+            }
+            if (p.lse != nullptr && row < p.Sq) {
+                const float m_use = (m == -INFINITY) ? 0.0f : m;
+                p.lse[(static_cast<size_t>(b) * p.H + h) * p.Sq + row] =
+                    (m_use + __log2f(l)) * 0.69314718055994531f;
+            }
+        }
+    }
+
+    // ------------------------------------------------ teardown
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        __syncwarp();
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace vdit

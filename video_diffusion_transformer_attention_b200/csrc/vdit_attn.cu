@@ -1,0 +1,247 @@
+// vdit_attn.cu -- host side of libvdit_attn.so: argument validation, TMA
+// tensor maps, launch, and the device status word.  The C ABI is declared in
+// include/vdit_attn.h; every entry point returns a status code and lets no
+// C++ exception escape.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "vdit_attn.h"
+#include "attn_fwd_sm100.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultWaitTimeoutNs = 2000000000ull;  // 2 s per barrier wait
+
+// ------------------------------------------------------------ argument checks
+
+struct Shape {
+    int B, H, Sq, Skv, D, mask_kind, chunk;
+};
+
+vdit_status check_shape(const Shape& s, bool check_scale, float scale) {
+    if (s.B < 0 || s.H < 0 || s.Sq < 0 || s.Skv < 1 || s.D < 1) return VDIT_ERR_INVALID_ARG;
+    if (s.mask_kind != VDIT_MASK_FULL && s.mask_kind != VDIT_MASK_BLOCK_CAUSAL && s.mask_kind != VDIT_MASK_CROSS)
+        return VDIT_ERR_INVALID_ARG;
+    if (s.D != vdit::kHeadDim) return VDIT_ERR_UNSUPPORTED;
+    if (s.mask_kind == VDIT_MASK_BLOCK_CAUSAL && (s.chunk < 1 || s.Sq != s.Skv)) return VDIT_ERR_INVALID_ARG;
+    if (s.B > 65535 || s.H > 65535) return VDIT_ERR_INVALID_ARG;
+    if (check_scale && !(std::isfinite(scale) && scale > 0.0f)) return VDIT_ERR_INVALID_ARG;
+    return VDIT_OK;
+}
+
+int grid_x(int Sq) { return (Sq + vdit::kQTiles * vdit::kBlockM - 1) / (vdit::kQTiles * vdit::kBlockM); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+// ------------------------------------------------------------ per-device setup
+
+struct DeviceState {
+    std::once_flag once;
+    vdit_status status = VDIT_ERR_CUDA;
+};
+DeviceState g_devices[kMaxDevices];
+
+void init_device(int dev, DeviceState* st) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        st->status = VDIT_ERR_CUDA;
+        return;
+    }
+    if (major != 10 || minor != 0) {
+        st->status = VDIT_ERR_UNSUPPORTED;
+        return;
+    }
+    if (cudaFuncSetAttribute(vdit::attn_fwd_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             vdit::kSmemBytes) != cudaSuccess) {
+        st->status = VDIT_ERR_CUDA;
+        return;
+    }
+    st->status = VDIT_OK;
+}
+
+vdit_status ensure_device(int* dev_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return VDIT_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return VDIT_ERR_UNSUPPORTED;
+    DeviceState* st = &g_devices[dev];
+    std::call_once(st->once, init_device, dev, st);
+    *dev_out = dev;
+    return st->status;
+}
+
+// ------------------------------------------------------------ TMA tensor maps
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};
+    PFN_cuTensorMapEncodeTiled_v12000 f = fn.load();
+    if (f == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        f = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        fn.store(f);
+    }
+    return f;
+}
+
+// [B][S][H][D] bf16 viewed as a 4-D tensor (D, H, S, B), innermost first; a
+// box is 64 head dims x 1 head x 128 tokens x 1 batch, 128-byte swizzled, so
+// each box lands as 128 rows of 128 bytes (one K-major / MN-major SW128 atom
+// column).  Rows past S read as zero.
+bool encode_bshd(CUtensorMap* map, const void* base, int B, int S, int H) {
+    PFN_cuTensorMapEncodeTiled_v12000 f = encode_fn();
+    if (f == nullptr) return false;
+    const cuuint64_t D = vdit::kHeadDim;
+    cuuint64_t dims[4] = {D, cuuint64_t(H), cuuint64_t(S), cuuint64_t(B)};
+    cuuint64_t strides[3] = {D * 2, cuuint64_t(H) * D * 2, cuuint64_t(S) * cuuint64_t(H) * D * 2};
+    cuuint32_t box[4] = {64, 1, cuuint32_t(vdit::kBlockM), 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = f(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+vdit_status launch(const void* q, const void* k, const void* v, void* o, float* lse, const Shape& s, float scale,
+                   cudaStream_t stream) {
+    int dev = 0;
+    vdit_status st = ensure_device(&dev);
+    if (st != VDIT_OK) return st;
+    CUtensorMap tq, tk, tv;
+    if (!encode_bshd(&tq, q, s.B, s.Sq, s.H) || !encode_bshd(&tk, k, s.B, s.Skv, s.H) ||
+        !encode_bshd(&tv, v, s.B, s.Skv, s.H))
+        return VDIT_ERR_CUDA;
+    vdit::FwdParams p{};
+    p.B = s.B;
+    p.H = s.H;
+    p.Sq = s.Sq;
+    p.Skv = s.Skv;
+    p.mask_kind = s.mask_kind;
+    p.chunk = s.mask_kind == VDIT_MASK_BLOCK_CAUSAL ? s.chunk : 1;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.timeout_ns = kDefaultWaitTimeoutNs;
+    dim3 grid(grid_x(s.Sq), s.H, s.B);
+    vdit::attn_fwd_sm100_kernel<<<grid, vdit::kNumThreads, vdit::kSmemBytes, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
+}
+
+vdit_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
+                     int Skv, int D, float scale, int mask_kind, int chunk_tokens, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+    (void)workspace;
+    (void)workspace_bytes;  // no shape needs a workspace in this version
+    const Shape s{B, H, Sq, Skv, D, mask_kind, chunk_tokens};
+    vdit_status st = check_shape(s, true, scale);
+    if (st != VDIT_OK) return st;
+    if (B == 0 || H == 0 || Sq == 0) return VDIT_OK;
+    if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return VDIT_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return VDIT_ERR_MISALIGNED;
+    const size_t row_bytes = size_t(H) * size_t(D) * 2;
+    const size_t q_bytes = size_t(B) * size_t(Sq) * row_bytes;
+    const size_t kv_bytes = size_t(B) * size_t(Skv) * row_bytes;
+    if (overlaps(o, q_bytes, q, q_bytes) || overlaps(o, q_bytes, k, kv_bytes) || overlaps(o, q_bytes, v, kv_bytes))
+        return VDIT_ERR_INVALID_ARG;
+    if (lse != nullptr) {
+        const size_t lse_bytes = size_t(B) * size_t(H) * size_t(Sq) * 4;
+        if (overlaps(lse, lse_bytes, o, q_bytes) || overlaps(lse, lse_bytes, q, q_bytes) ||
+            overlaps(lse, lse_bytes, k, kv_bytes) || overlaps(lse, lse_bytes, v, kv_bytes))
+            return VDIT_ERR_INVALID_ARG;
+    }
+    return launch(q, k, v, o, lse, s, scale, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+int vdit_abi_version(void) { return VDIT_ATTN_ABI_VERSION; }
+
+const char* vdit_status_string(int status) {
+    switch (status) {
+        case VDIT_OK: return "VDIT_OK";
+        case VDIT_ERR_INVALID_ARG: return "VDIT_ERR_INVALID_ARG";
+        case VDIT_ERR_UNSUPPORTED: return "VDIT_ERR_UNSUPPORTED";
+        case VDIT_ERR_MISALIGNED: return "VDIT_ERR_MISALIGNED";
+        case VDIT_ERR_CUDA: return "VDIT_ERR_CUDA";
+        case VDIT_ERR_TIMEOUT: return "VDIT_ERR_TIMEOUT";
+        case VDIT_ERR_WORKSPACE: return "VDIT_ERR_WORKSPACE";
+        default: return "VDIT_ERR_UNKNOWN";
+    }
+}
+
+vdit_status vdit_attn_plan(int B, int H, int Sq, int Skv, int D, int mask_kind, int chunk_tokens,
+                           size_t* workspace_bytes, int* grid_ctas) {
+    try {
+        const Shape s{B, H, Sq, Skv, D, mask_kind, chunk_tokens};
+        vdit_status st = check_shape(s, false, 1.0f);
+        if (st != VDIT_OK) return st;
+        if (workspace_bytes == nullptr) return VDIT_ERR_INVALID_ARG;
+        *workspace_bytes = 0;
+        if (grid_ctas != nullptr) {
+            const long long n = (B == 0 || H == 0 || Sq == 0) ? 0 : (long long)grid_x(Sq) * H * B;
+            *grid_ctas = n > 0x7fffffffLL ? 0x7fffffff : int(n);
+        }
+        return VDIT_OK;
+    } catch (...) {
+        return VDIT_ERR_INVALID_ARG;
+    }
+}
+
+vdit_status vdit_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
+                          int Skv, int D, float scale, int mask_kind, int chunk_tokens, void* stream) {
+    try {
+        return fwd_impl(q, k, v, o, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, nullptr, 0, stream);
+    } catch (...) {
+        return VDIT_ERR_CUDA;
+    }
+}
+
+vdit_status vdit_attn_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                             int Sq, int Skv, int D, float scale, int mask_kind, int chunk_tokens, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+    try {
+        return fwd_impl(q, k, v, o, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, workspace,
+                        workspace_bytes, stream);
+    } catch (...) {
+        return VDIT_ERR_CUDA;
+    }
+}
+
+vdit_status vdit_get_device_status(void* stream, uint32_t* detail) {
+    try {
+        if (detail != nullptr) *detail = 0;
+        if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return VDIT_ERR_CUDA;
+        uint32_t word = 0;
+        if (cudaMemcpyFromSymbol(&word, vdit::g_status_word, sizeof(word)) != cudaSuccess) return VDIT_ERR_CUDA;
+        if (word != 0) {
+            const uint32_t zero = 0;
+            if (cudaMemcpyToSymbol(vdit::g_status_word, &zero, sizeof(zero)) != cudaSuccess) return VDIT_ERR_CUDA;
+        }
+        if (detail != nullptr) *detail = word;
+        return (word & vdit::kStatusTimeout) ? VDIT_ERR_TIMEOUT : VDIT_OK;
+    } catch (...) {
+        return VDIT_ERR_CUDA;
+    }
+}
+
+}  // extern "C"
