@@ -1,0 +1,368 @@
+#!/usr/bin/env python
+"""Benchmark of the bf16 video-DiT attention forward on B200.
+
+One step = one pass of the whole hot path over the 720p Wan2.1-14B workload:
+self-attention (B=1, H=40, Sq=Skv=75,600, D=128, full mask) followed by
+cross-attention of the same queries to 512 text tokens.  Inputs are seeded
+synthetic tensors (see video_diffusion_transformer_attention_b200/workloads.py),
+far larger than L2, resident in HBM before the timed region.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl vdit|reference]
+
+For N > 1 launch under torch.distributed.run: every rank runs the full
+workload on its own GPU (independent problems, no collective on the data
+path; "weak" scaling); the time is the max over ranks.  Rank 0 prints one JSON
+line.  ``--impl reference`` times the fp64 CPU oracle on a bounded row sample
+of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from video_diffusion_transformer_attention_b200 import flops as fl  # noqa: E402
+from video_diffusion_transformer_attention_b200 import workloads as wl  # noqa: E402
+
+WORKLOAD = "wan21_14b_720p"
+METRIC = "bf16 video-DiT attention fwd TFLOP/s & % of B200 BF16 peak; ms at S=75600"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DATASHEET_BF16_TFLOPS = 2250.0
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(name):
+    w = wl.WORKLOADS[name]
+    desc = "; ".join(
+        f"{c.name}: B={c.B} H={c.H} Sq={c.Sq} Skv={c.Skv} D={c.D} mask="
+        f"{['full', 'block_causal', 'cross'][c.mask_kind]}" + (f" chunk={c.chunk_tokens}" if c.chunk_tokens else "")
+        for c in w.calls)
+    return w, desc
+
+
+def call_inputs(inp, call):
+    if call.mask_kind == wl.MASK_CROSS:
+        return inp["q"], inp["k_text"], inp["v_text"]
+    return inp["q"], inp["k"], inp["v"]
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples taken while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle legs
+
+def oracle_sample(inp, w, seconds_budget=20.0, seed=0):
+    """Time the fp64 oracle on a bounded row sample of every call; TFLOP/s."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    total_flops, total_time, parts = 0.0, 0.0, []
+    for call in w.calls:
+        q, k, v = call_inputs(inp, call)
+        qb, kb, vb = wl.bf16_bits(q), wl.bf16_bits(k), wl.bf16_bits(v)
+        # an equal share of the budget per call, at about 0.5 GFLOP/s per core
+        # for this plain fp64 loop
+        flops_row = 4.0 * call.D * call.Skv
+        n = int(max(8, min(call.B * call.H * call.Sq,
+                          seconds_budget / len(w.calls) * 0.5e9 * oracle.max_threads() / flops_row)))
+        rows = np.stack([rng.integers(0, call.B, n), rng.integers(0, call.H, n),
+                         rng.integers(0, call.Sq, n)], axis=1)
+        t0 = time.perf_counter()
+        oracle.attention(qb, kb, vb, call.scale, call.mask_kind, call.chunk_tokens, rows=rows)
+        dt = time.perf_counter() - t0
+        f = flops_row * n
+        total_flops += f
+        total_time += dt
+        parts.append(f"{call.name}: {n} rows x {call.Skv} keys")
+    return total_flops, total_time, "; ".join(parts)
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    w, desc = workload_config(args.workload)
+    inp = wl.workload_inputs(args.workload)
+    times, flops_done = [], []
+    sample = ""
+    # keep the whole --steps/--warmup run within a few minutes of CPU time
+    budget = min(args.reference_seconds, 150.0 / max(1, args.warmup + args.steps))
+    for s in range(args.warmup + args.steps):
+        f, t, sample = oracle_sample(inp, w, seconds_budget=budget, seed=s)
+        if s >= args.warmup:
+            times.append(t)
+            flops_done.append(f)
+    value = sum(flops_done) / sum(times) / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{args.workload} ({desc})", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU leg
+
+def run_vdit(args):
+    from video_diffusion_transformer_attention_b200 import binding as vb
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    vb.lib()
+    w, desc = workload_config(args.workload)
+    inp_cpu = wl.workload_inputs(args.workload)
+    inp = {k: v.to(dev) for k, v in inp_cpu.items()}
+    outs = []
+    for call in w.calls:
+        outs.append((torch.empty((call.B, call.Sq, call.H, call.D), dtype=torch.bfloat16, device=dev),
+                     torch.empty((call.B, call.H, call.Sq), dtype=torch.float32, device=dev)))
+    stream = torch.cuda.Stream(device=dev)
+    sptr = int(stream.cuda_stream)
+    flops_per_call = [fl.attn_flops(c) for c in w.calls]
+    step_flops = sum(flops_per_call)
+
+    def launch(i, call, q, k, v, o, lse):
+        vb.vdit_attn_fwd(q, k, v, o, lse, call.B, call.H, call.Sq, call.Skv, call.D, call.scale,
+                         call.mask_kind, call.chunk_tokens, sptr)
+
+    def step(events=None):
+        for i, call in enumerate(w.calls):
+            q, k, v = call_inputs(inp, call)
+            if events is not None:
+                events[i][0].record(stream)
+            launch(i, call, q, k, v, *outs[i])
+            if events is not None:
+                events[i][1].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    st, word = vb.vdit_get_device_status(sptr)
+    if st != vb.VDIT_OK:
+        raise SystemExit(f"device status after warm-up: {vb.vdit_status_string(st)} ({word:#x})")
+
+    per_call_events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                        for _ in w.calls] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(per_call_events[s])
+    t_end.record(stream)
+    stream.synchronize()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end)
+    call_ms = [statistics.mean(per_call_events[s][i][0].elapsed_time(per_call_events[s][i][1])
+                               for s in range(args.steps)) for i in range(len(w.calls))]
+    st, word = vb.vdit_get_device_status(sptr)
+    if st != vb.VDIT_OK:
+        raise SystemExit(f"device status after timing: {vb.vdit_status_string(st)} ({word:#x})")
+    ms_max = ms
+    if dist is not None:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    ms_per_step = ms_max / args.steps
+    value = world * step_flops * args.steps / (ms_max * 1e-3) / 1e12
+
+    # ---- end to end through the public API, host buffers in and out
+    e2e = None
+    if args.e2e_steps > 0:
+        host_in = {k: v.pin_memory() for k, v in inp_cpu.items()}
+        host_out = [(torch.empty(o.shape, dtype=o.dtype).pin_memory(), torch.empty(l.shape, dtype=l.dtype).pin_memory())
+                    for o, l in outs]
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        d2h = sum(o.numel() * o.element_size() + l.numel() * l.element_size() for o, l in host_out)
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                for k_, v_ in host_in.items():
+                    inp[k_].copy_(v_, non_blocking=True)
+                step()
+                for (o, l), (ho, hl) in zip(outs, host_out):
+                    ho.copy_(o, non_blocking=True)
+                    hl.copy_(l, non_blocking=True)
+
+        e2e_step()
+        stream.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        stream.synchronize()
+        barrier()
+        e_ms = e0.elapsed_time(e1)
+        if dist is not None:
+            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * step_flops * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps}
+
+    line = None
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        # the self-attention launch dominates the step
+        dom = 0
+        achieved = flops_per_call[dom] / (call_ms[dom] * 1e-3) / 1e12
+        peak_sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        cross = w.calls[1] if len(w.calls) > 1 else None
+        calls = []
+        for i, c in enumerate(w.calls):
+            calls.append({"call": c.name, "ms": call_ms[i], "tflops": flops_per_call[i] / (call_ms[i] * 1e-3) / 1e12,
+                          "hbm_gbs": fl.attn_min_bytes(c) / (call_ms[i] * 1e-3) / 1e9})
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{args.workload} ({desc})", "l2": "inputs larger than L2 (3.1 GB per step)",
+                       "parallelism": f"independent replicas x{world} (no collective)"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_sustained, "unit": "TFLOP/s",
+                         "frac": achieved / peak_sustained, "traffic": None,
+                         "kernel": "attn_fwd_sm100_kernel (self-attention launch)",
+                         "peak_kind": f"{peak_src} sustained bf16 (cuBLAS, power-capped)",
+                         "frac_of_burst": achieved / peak_burst,
+                         "frac_of_datasheet": achieved / DATASHEET_BF16_TFLOPS},
+            "calls": calls,
+            "clocks": clk,
+            "e2e": e2e,
+            "gpu_launches": len(w.calls) * args.steps,
+        }
+        if cross is not None:
+            line["roofline"]["cross_hbm_frac"] = calls[1]["hbm_gbs"] / float(peaks.get("hbm_gbs", 6650.0))
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        f, t, sample = oracle_sample(inp_cpu, w, seconds_budget=args.reference_seconds)
+        line["cpu_baseline"] = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(),
+                                "kind": "oracle", "sample": sample, "seconds": t}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("vdit", "reference"), default="vdit")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--reference-seconds", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "vdit":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_vdit(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

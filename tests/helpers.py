@@ -4,7 +4,8 @@ The checker holds the graded bars: max|err| <= 1e-2 and mean|err| <= 1e-3 on
 bf16 O against the fp64 oracle rounded to bf16, relative error <= 1e-3 on the
 fp32 LSE (relative to max(|LSE|, 1)).  Because attention outputs shrink like sqrt(e / Skv) at long
 sequences, it adds two scale-aware bars that an all-zero or shuffled O cannot
-pass: max|err| / rms(O_ref) <= 2e-2 per (b, h), and cosine(O, O_ref) >= 0.9999.
+pass: rms(err) / rms(O_ref) <= 1e-2 per (b, h), and cosine(O, O_ref) >= 0.9999.
+(bf16 rounding of O alone contributes about 2^-9 / sqrt(3) ~ 1e-3 to the first.)
 """
 import numpy as np
 import torch
@@ -12,7 +13,7 @@ import torch
 MAX_ABS = 1e-2
 MEAN_ABS = 1e-3
 LSE_REL = 1e-3
-REL_TO_RMS = 2e-2
+REL_RMS_ERR = 1e-2
 MIN_COSINE = 0.9999
 
 
@@ -48,8 +49,9 @@ def check_parity(o_gpu, o_ref, lse_gpu, lse_ref, group_rows=None, label=""):
     worst_rel = 0.0
     for g in groups:
         rms = float(np.sqrt(np.mean(o_ref[g] ** 2)))
-        worst_rel = max(worst_rel, float(err[g].max()) / max(rms, 1e-30))
-    res["max_rel_rms"] = worst_rel
+        rms_err = float(np.sqrt(np.mean(err[g] ** 2)))
+        worst_rel = max(worst_rel, rms_err / max(rms, 1e-30))
+    res["rel_rms_err"] = worst_rel
     a, b = o_gpu.ravel(), np.asarray(o_ref, dtype=np.float64).ravel()
     res["cosine"] = float(a @ b / max(np.linalg.norm(a) * np.linalg.norm(b), 1e-300))
     if lse_gpu is not None:
@@ -59,7 +61,7 @@ def check_parity(o_gpu, o_ref, lse_gpu, lse_ref, group_rows=None, label=""):
         # sequence with small logits) is held to 1e-3 absolute instead
         res["lse_rel"] = float(np.max(np.abs(lg - lr) / np.maximum(np.abs(lr), 1.0)))
     ok = (res["max_abs"] <= MAX_ABS and res["mean_abs"] <= MEAN_ABS
-          and res["max_rel_rms"] <= REL_TO_RMS and res["cosine"] >= MIN_COSINE
+          and res["rel_rms_err"] <= REL_RMS_ERR and res["cosine"] >= MIN_COSINE
           and (lse_gpu is None or res["lse_rel"] <= LSE_REL))
     res["ok"] = bool(ok)
     res["label"] = label
