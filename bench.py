@@ -178,6 +178,22 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------------------ rank helpers
+
+def reduce_max(value, dist=None, device="cpu"):
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    if dist is None:
+        return float(value)
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world, step_flops, steps, ms):
+    """Whole-job throughput: every rank ran `steps` steps of `step_flops` in `ms`."""
+    return world * step_flops * steps / (ms * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ GPU leg
 
 def run_vdit(args):
@@ -256,13 +272,9 @@ def run_vdit(args):
     st, word = vb.vdit_get_device_status(sptr)
     if st != vb.VDIT_OK:
         raise SystemExit(f"device status after timing: {vb.vdit_status_string(st)} ({word:#x})")
-    ms_max = ms
-    if dist is not None:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = reduce_max(ms, dist, dev)
     ms_per_step = ms_max / args.steps
-    value = world * step_flops * args.steps / (ms_max * 1e-3) / 1e12
+    value = job_tflops(world, step_flops, args.steps, ms_max)
 
     # ---- end to end through the public API, host buffers in and out
     e2e = None
@@ -292,12 +304,8 @@ def run_vdit(args):
         e1.record(stream)
         stream.synchronize()
         barrier()
-        e_ms = e0.elapsed_time(e1)
-        if dist is not None:
-            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * step_flops * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e_ms = reduce_max(e0.elapsed_time(e1), dist, dev)
+        e2e = {"value": job_tflops(world, step_flops, args.e2e_steps, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps}
 
