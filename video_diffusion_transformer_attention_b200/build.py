@@ -7,6 +7,7 @@
 from __future__ import annotations
 
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -41,20 +42,43 @@ def stale() -> bool:
     return any(os.path.getmtime(f) > t for f in SOURCES + HEADERS)
 
 
+def _launch_regs_expected() -> int:
+    src = open(os.path.join(CSRC, "attn_fwd_sm100.cuh")).read()
+    return int(re.search(r"kLaunchRegs\s*=\s*(\d+)", src).group(1))
+
+
+def check_launch_registers(ptxas_log: str) -> int:
+    """The forward kernel re-splits its registers with setmaxnreg, which is only
+    safe if ptxas allocated exactly kLaunchRegs a thread at launch; a smaller
+    allocation would leave setmaxnreg.inc waiting forever.  Returns the count."""
+    m = re.search(r"Compiling entry function '\w*attn_fwd_sm100_kernel\w*'.*?Used (\d+) registers",
+                  ptxas_log, flags=re.S)
+    if m is None:
+        raise RuntimeError("could not find the forward kernel's register count in the ptxas output")
+    used, expected = int(m.group(1)), _launch_regs_expected()
+    if used != expected:
+        raise RuntimeError(f"attn_fwd_sm100_kernel allocates {used} registers a thread, "
+                           f"the setmaxnreg split assumes {expected}")
+    return used
+
+
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     if not force and not stale():
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC,
+    cmd = [nvcc(), "-Xptxas=-v", *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC,
            os.path.join(CSRC, "vdit_attn.cu"), "-o", tmp]
-    if verbose_ptxas:
-        cmd.insert(1, "-Xptxas=-v")
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
         raise RuntimeError("nvcc failed building libvdit_attn.so")
     if verbose_ptxas:
         sys.stderr.write(res.stderr)
+    try:
+        check_launch_registers(res.stderr)
+    except RuntimeError:
+        os.unlink(tmp)
+        raise
     os.replace(tmp, LIB)
     return LIB
 

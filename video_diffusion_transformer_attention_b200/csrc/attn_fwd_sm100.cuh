@@ -13,15 +13,24 @@
 // the running row maximum and row sum kept per query row ("VC-Attention"
 // (aikraft.ru), section 02, Restore step: the online softmax already holds
 // the row sum).  The exp + cast between the two products is the long pole on
-// B200 (same page, section 01), so the softmax runs in two warpgroups that
-// alternate with the tensor core: while warpgroup 0 exponentiates tile 0,
-// the tensor core computes P_1 V and S_1 for tile 1, and vice versa.
+// B200 (same page, section 01), so:
+//   * the softmax runs in two warpgroups that alternate with the tensor core:
+//     while warpgroup 0 exponentiates tile 0, the tensor core computes P_1 V
+//     and S_1 for tile 1, and vice versa;
+//   * P is handed over in two 64-key halves, so O_t += P_t V starts on keys
+//     0-63 while keys 64-127 are still being exponentiated;
+//   * the scale-and-subtract and the row sum run as packed fp32x2 ops, so the
+//     issue slots left over around MUFU ex2 stay free for the other warps.
 //
-// Roles (320 threads):
-//   warps 0-3  softmax + correction + epilogue of query tile 0
-//   warps 4-7  softmax + correction + epilogue of query tile 1
-//   warp  8    TMA producer (Q once, then K_j, V_j into a 4-slot ring)
-//   warp  9    TMEM allocator and single-thread tcgen05.mma issuer
+// Roles (384 threads, three warpgroups):
+//   warps 0-3   softmax + correction + epilogue of query tile 0
+//   warps 4-7   softmax + correction + epilogue of query tile 1
+//   warp  8     TMA producer (Q once, then K_j, V_j into a 4-slot ring)
+//   warp  9     TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 10-11 idle
+// The kernel is launched at 168 registers a thread (384 x 168 = 64,512); the
+// softmax warpgroups then raise theirs to 208 and the third lowers its to 88
+// (2 x 128 x 208 + 128 x 88 = 64,512, the same total).
 //
 // TMEM (512 columns x 128 lanes, fp32): S_0 [0,128), S_1 [128,256),
 // O_0 [256,384), O_1 [384,512).  P_t (bf16, two per column) overwrites the
@@ -46,9 +55,14 @@ constexpr int kQTiles = 2;     // query tiles per CTA
 constexpr int kStages = 4;     // K/V ring slots (each holds one K or one V tile)
 constexpr int kTileBytes = kBlockM * kHeadDim * 2;  // 32 KB
 constexpr int kHalfBytes = kTileBytes / 2;          // 128 rows x 64 bf16, 128B-swizzled
-constexpr int kNumThreads = 320;
+constexpr int kNumThreads = 384;
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kLaunchRegs = 168;    // ptxas allocation at launch (checked by the build)
+constexpr int kSoftmaxRegs = 208;   // after setmaxnreg.inc in warpgroups 0 and 1
+constexpr int kControlRegs = 88;    // after setmaxnreg.dec in warpgroup 2
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kNumThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 
@@ -67,7 +81,7 @@ struct __align__(8) Barriers {
     uint64_t kv_full[kStages];
     uint64_t kv_empty[kStages];
     uint64_t s_full[kQTiles];
-    uint64_t p_full[kQTiles];
+    uint64_t p_full[kQTiles][2];  // P keys 0-63 / 64-127 of tile t in TMEM
     uint64_t o_full[kQTiles];
     uint64_t drain;  // MMA issuer's own completion barrier on the abort path
     uint32_t tmem_base;
@@ -139,31 +153,56 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 
 // ---------------------------------------------------------------- MMA helpers
 
+// The MMA issuer keeps one descriptor per operand base and advances it by
+// adding (byte offset >> 4) to the start-address field: every operand offset
+// used below stays inside the 14-bit field, so the add never carries into the
+// leading-byte-offset bits.
+//
 // S[128 x 128] = Q_tile[128 x 128] * K_tile[128 x 128]^T, both K-major with
 // 128B swizzle, each stored as two 16 KB halves (head dims 0-63 and 64-127).
 // K = 16 per instruction: 4 steps of 32 bytes inside a half, then the next half.
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc) {
     constexpr uint32_t idesc = make_idesc_bf16(false);
 #pragma unroll
     for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-        const uint32_t off = uint32_t(kk >> 2) * kHalfBytes + uint32_t(kk & 3) * 32u;
-        umma_ss(d_tmem, smem_desc_sw128(q_smem + off, 16, 1024), smem_desc_sw128(k_smem + off, 16, 1024),
-                idesc, kk > 0 ? 1u : 0u);
+        const uint64_t off = (uint64_t(kk >> 2) * kHalfBytes + uint64_t(kk & 3) * 32u) >> 4;
+        umma_ss(d_tmem, q_desc + off, k_desc + off, idesc, kk > 0 ? 1u : 0u);
     }
 }
 
-// O[128 x 128] (+)= P[128 x 128 keys] * V_tile[128 keys x 128].  P comes from
-// TMEM (two bf16 per column, 8 columns per K = 16 step).  V is the B operand
-// in MN-major form: head dim is contiguous; 64-dim halves are 16 KB apart
-// (leading byte offset), 8-key row groups 1 KB apart (stride byte offset),
-// and each 16-key step advances 16 rows = 2 KB.
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem,
-                                         bool accumulate) {
+// O[128 x 128] (+)= P[128 x keys] * V_tile[keys x 128] for the 64 keys of
+// `half`.  P comes from TMEM (two bf16 per column, 8 columns per K = 16
+// step).  V is the B operand in MN-major form: head dim is contiguous; 64-dim
+// halves are 16 KB apart (leading byte offset), 8-key row groups 1 KB apart
+// (stride byte offset), and each 16-key step advances 16 rows = 2 KB.
+__device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, uint64_t v_desc, int half,
+                                              bool accumulate) {
     constexpr uint32_t idesc = make_idesc_bf16(true);
 #pragma unroll
-    for (int kk = 0; kk < kBlockN / 16; ++kk) {
-        umma_ts(d_tmem, p_tmem + uint32_t(kk) * 8u, smem_desc_sw128(v_smem + uint32_t(kk) * 2048u, kHalfBytes, 1024),
-                idesc, (accumulate || kk > 0) ? 1u : 0u);
+    for (int i = 0; i < kBlockN / 32; ++i) {
+        const int kk = half * (kBlockN / 32) + i;
+        umma_ts(d_tmem, p_tmem + uint32_t(kk) * 8u, v_desc + uint64_t(kk) * (2048u >> 4), idesc,
+                (accumulate || kk > 0) ? 1u : 0u);
+    }
+}
+
+// ---------------------------------------------------------------- softmax pieces
+
+// Exponentiate 32 logits (one TMEM chunk of the row): x = s*scale*log2e - m as
+// packed fp32x2 FMAs, 2^x on MUFU (ex2.approx), the fp32 row sum as packed
+// adds into four accumulators, and bf16x2 packing of the pairs into pk[0..15].
+// (Taking part of the exponentials on the FMA pipe with a polynomial was
+// measured slower than MUFU alone at this occupancy, so every pair uses MUFU.)
+__device__ __forceinline__ void exp_chunk(const uint32_t (&s)[32], uint64_t scale2, uint64_t negm2,
+                                          uint32_t (&pk)[16], uint64_t (&lsum)[4]) {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        float x0, x1;
+        ffma2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1]), scale2, negm2, x0, x1);
+        const float p0 = ex2_approx(x0);
+        const float p1 = ex2_approx(x1);
+        fadd2_acc(lsum[k & 3], p0, p1);
+        pk[k] = pack_bf16x2(p0, p1);
     }
 }
 
@@ -188,7 +227,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         for (int t = 0; t < kQTiles; ++t) {
             mbar_init(smem_addr(&bars->q_full[t]), 1);
             mbar_init(smem_addr(&bars->s_full[t]), 1);
-            mbar_init(smem_addr(&bars->p_full[t]), 4 * 32);
+            mbar_init(smem_addr(&bars->p_full[t][0]), 4);  // one elected arrive per softmax warp
+            mbar_init(smem_addr(&bars->p_full[t][1]), 4);
             mbar_init(smem_addr(&bars->o_full[t]), 1);
         }
         for (int s = 0; s < kStages; ++s) {
@@ -226,9 +266,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const uint32_t sQ = smem_addr(smem + kSmemQ);
     const uint32_t sKV = smem_addr(smem + kSmemKV);
 
-    if (warp == kLoadWarp) {
-        // ------------------------------------------------ TMA producer
-        if (lane == 0) {
+    if (warp >= 8) {
+        setmaxnreg_dec<kControlRegs>();
+        if (warp == kLoadWarp && lane == 0) {
+            // ------------------------------------------------ TMA producer
             for (int t = 0; t < kQTiles; ++t) {
                 const uint32_t bar = smem_addr(&bars->q_full[t]);
                 mbar_arrive_expect_tx(bar, kTileBytes);
@@ -248,59 +289,61 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 tma_load_4d(sKV + slot * kTileBytes, map, full, 0, h, row, b);
                 tma_load_4d(sKV + slot * kTileBytes + kHalfBytes, map, full, 64, h, row, b);
             }
-        }
-    } else if (warp == kMmaWarp) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
+        } else if (warp == kMmaWarp && lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            const uint32_t tS[2] = {tmem, tmem + 128};
+            const uint32_t tO[2] = {tmem + 256, tmem + 384};
+            // descriptor bases: Q tiles (K-major), ring slots as K (K-major) and as V (MN-major)
+            const uint64_t q_desc[2] = {smem_desc_sw128(sQ, 16, 1024), smem_desc_sw128(sQ + kTileBytes, 16, 1024)};
+            const uint64_t k_desc0 = smem_desc_sw128(sKV, 16, 1024);
+            const uint64_t v_desc0 = smem_desc_sw128(sKV, kHalfBytes, 1024);
+            constexpr uint64_t kSlotStep = kTileBytes >> 4;
             bool ok = bounded_wait(smem_addr(&bars->q_full[0]), 0, abort_flag, p.timeout_ns, kSiteMma) &&
                       bounded_wait(smem_addr(&bars->q_full[1]), 0, abort_flag, p.timeout_ns, kSiteMma);
             // prologue: S_0 and S_1 against K_0
-            int k_slot = 0;
             if (ok) ok = bounded_wait(smem_addr(&bars->kv_full[0]), 0, abort_flag, p.timeout_ns, kSiteMma);
             if (ok) {
                 tc_fence_after_sync();
-                issue_qk(tS0, sQ, sKV);
+                issue_qk(tS[0], q_desc[0], k_desc0);
                 umma_commit(smem_addr(&bars->s_full[0]));
-                issue_qk(tS1, sQ + kTileBytes, sKV);
+                issue_qk(tS[1], q_desc[1], k_desc0);
                 umma_commit(smem_addr(&bars->s_full[1]));
                 umma_commit(smem_addr(&bars->kv_empty[0]));
             }
+            // steady state, per key tile j:
+            //   PV0(j) [two halves]  S0(j+1)  PV1(j) [two halves]  S1(j+1)
             for (int j = 0; ok && j < n_kv; ++j) {
                 const int uv = 2 * j + 1;
                 const int v_slot = uv % kStages;
-                ok = bounded_wait(smem_addr(&bars->kv_full[v_slot]), uint32_t(uv / kStages) & 1u, abort_flag,
-                                  p.timeout_ns, kSiteMma) &&
-                     bounded_wait(smem_addr(&bars->p_full[0]), uint32_t(j) & 1u, abort_flag, p.timeout_ns,
-                                  kSiteMma);
-                if (!ok) break;
-                tc_fence_after_sync();
-                issue_pv(tO0, tS0, sKV + v_slot * kTileBytes, j > 0);
+                const int uk = 2 * (j + 1);
+                const int k_slot = uk % kStages;
+                const uint32_t ph = uint32_t(j) & 1u;
                 const bool more = (j + 1) < n_kv;
-                if (more) {
-                    const int uk = 2 * (j + 1);
-                    k_slot = uk % kStages;
-                    ok = bounded_wait(smem_addr(&bars->kv_full[k_slot]), uint32_t(uk / kStages) & 1u,
-                                      abort_flag, p.timeout_ns, kSiteMma);
+                ok = bounded_wait(smem_addr(&bars->kv_full[v_slot]), uint32_t(uv / kStages) & 1u, abort_flag,
+                                  p.timeout_ns, kSiteMma);
+                for (int t = 0; ok && t < kQTiles; ++t) {
+                    for (int hf = 0; ok && hf < 2; ++hf) {
+                        ok = bounded_wait(smem_addr(&bars->p_full[t][hf]), ph, abort_flag, p.timeout_ns, kSiteMma);
+                        if (ok) {
+                            tc_fence_after_sync();
+                            issue_pv_half(tO[t], tS[t], v_desc0 + uint64_t(v_slot) * kSlotStep, hf, j > 0);
+                        }
+                    }
                     if (!ok) break;
-                    tc_fence_after_sync();
-                    issue_qk(tS0, sQ, sKV + k_slot * kTileBytes);
-                    umma_commit(smem_addr(&bars->s_full[0]));
-                } else {
-                    umma_commit(smem_addr(&bars->o_full[0]));
-                }
-                ok = bounded_wait(smem_addr(&bars->p_full[1]), uint32_t(j) & 1u, abort_flag, p.timeout_ns,
-                                  kSiteMma);
-                if (!ok) break;
-                tc_fence_after_sync();
-                issue_pv(tO1, tS1, sKV + v_slot * kTileBytes, j > 0);
-                umma_commit(smem_addr(&bars->kv_empty[v_slot]));
-                if (more) {
-                    issue_qk(tS1, sQ + kTileBytes, sKV + k_slot * kTileBytes);
-                    umma_commit(smem_addr(&bars->s_full[1]));
-                    umma_commit(smem_addr(&bars->kv_empty[k_slot]));
-                } else {
-                    umma_commit(smem_addr(&bars->o_full[1]));
+                    if (t == 1) umma_commit(smem_addr(&bars->kv_empty[v_slot]));
+                    if (more) {
+                        if (t == 0) {
+                            ok = bounded_wait(smem_addr(&bars->kv_full[k_slot]), uint32_t(uk / kStages) & 1u,
+                                              abort_flag, p.timeout_ns, kSiteMma);
+                            if (!ok) break;
+                            tc_fence_after_sync();
+                        }
+                        issue_qk(tS[t], q_desc[t], k_desc0 + uint64_t(k_slot) * kSlotStep);
+                        umma_commit(smem_addr(&bars->s_full[t]));
+                        if (t == 1) umma_commit(smem_addr(&bars->kv_empty[k_slot]));
+                    } else {
+                        umma_commit(smem_addr(&bars->o_full[t]));
+                    }
                 }
             }
             if (!ok) {
@@ -315,6 +358,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         }
     } else {
         // ------------------------------------------------ softmax warpgroups
+        setmaxnreg_inc<kSoftmaxRegs>();
         const int t = warp >> 2;        // query tile
         const int quarter = warp & 3;   // TMEM lane quarter this warp may access
         const int row_in_tile = quarter * 32 + lane;
@@ -323,7 +367,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const uint32_t tS = tmem + lane_bits + uint32_t(t) * 128u;
         const uint32_t tO = tmem + lane_bits + 256u + uint32_t(t) * 128u;
         const uint32_t s_full = smem_addr(&bars->s_full[t]);
-        const uint32_t p_full = smem_addr(&bars->p_full[t]);
 
         int kv_lim = p.Skv;  // keys [0, kv_lim) are allowed for this row
         if (p.mask_kind == kMaskBlockCausal) {
@@ -353,11 +396,18 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     for (int i = 0; i < 32; ++i)
                         if (c * 32 + i >= lim) s[c][i] = __float_as_uint(-INFINITY);
             }
-            float mx = -INFINITY;
+            // row max: eight independent 3-input max chains, then combine
+            float mxc[8];
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+            for (int g = 0; g < 8; ++g) {
+                const uint32_t* v = &s[g >> 1][(g & 1) * 16];
+                float a = fmaxf(__uint_as_float(v[0]), __uint_as_float(v[1]));
 #pragma unroll
-                for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(s[c][i]));
+                for (int i = 2; i < 16; i += 2) a = fmax3(a, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+                mxc[g] = a;
+            }
+            const float mx = fmax3(fmax3(mxc[0], mxc[1], mxc[2]), fmax3(mxc[3], mxc[4], mxc[5]),
+                                   fmaxf(mxc[6], mxc[7]));
             const float m_tile = mx * scale_log2;
 
             float alpha = 1.0f;
@@ -370,23 +420,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 l *= alpha;
                 rescale = true;
             }
-            const float m_use = (m == -INFINITY) ? 0.0f : m;
-            // P = exp2(S * scale*log2e - m) with the row sum in fp32; each pair
-            // is packed to bf16x2 into the register slot it has just consumed,
-            // and 16 packed columns at a time go back over S in TMEM.
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-#pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(s[c][i]), scale_log2, -m_use));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(s[c][i + 1]), scale_log2, -m_use));
-                    l += p0 + p1;
-                    s[c][i / 2] = pack_bf16x2(p0, p1);
-                }
-                tmem_st16(tS + uint32_t(c) * 16u, s[c]);
-            }
             if (__any_sync(0xffffffffu, rescale)) {
-                // O_t holds sum_k P_k V_k at the old reference: bring it to the new one.
+                // O_t holds sum_k P_k V_k at the old reference: bring it to the
+                // new one before any half of this tile's P is released.
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t o[32];
@@ -397,9 +433,34 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     tmem_st32(tO + uint32_t(c) * 32u, o);
                 }
             }
-            tmem_st_wait();
-            tc_fence_before_sync();
-            mbar_arrive(p_full);
+            const float m_use = (m == -INFINITY) ? 0.0f : m;
+            // P = exp2(S * scale*log2e - m) in two 64-key halves; each half goes
+            // to TMEM (over S columns already read) and is released to the MMA
+            // issuer on its own barrier.
+            const uint64_t scale2 = pack_f32x2(scale_log2, scale_log2);
+            const uint64_t negm2 = pack_f32x2(-m_use, -m_use);
+            uint64_t lsum[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c = hf * 2 + cc;
+                    uint32_t pk[16];
+                    exp_chunk(s[c], scale2, negm2, pk, lsum);
+                    tmem_st16(tS + uint32_t(c) * 16u, pk);
+                }
+                tmem_st_wait();
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&bars->p_full[t][hf]));
+            }
+            {
+                float part = 0.0f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    part += __uint_as_float(uint32_t(lsum[q])) + __uint_as_float(uint32_t(lsum[q] >> 32));
+                l += part;
+            }
         }
 
         if (ok) ok = warp_wait(smem_addr(&bars->o_full[t]), 0, abort_flag, p.timeout_ns, kSiteSoftmax);

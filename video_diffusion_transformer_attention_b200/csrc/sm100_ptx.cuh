@@ -175,12 +175,59 @@ __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- registers
+
+// Warp-granular register re-split between warpgroups (all warps of a
+// warpgroup execute the same one).
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- math
 
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 3-input maximum (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+__host__ __device__ constexpr uint64_t pack_f32x2_bits(uint32_t lo, uint32_t hi) {
+    return (uint64_t(hi) << 32) | uint64_t(lo);
+}
+
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+    return pack_f32x2_bits(__float_as_uint(lo), __float_as_uint(hi));
+}
+
+// (d0, d1) = (a0, a1) * b2 + c2, two fp32 FMAs in one instruction.
+__device__ __forceinline__ void ffma2(float a0, float a1, uint64_t b2, uint64_t c2, float& d0, float& d1) {
+    asm("{\n\t.reg .b64 a, d;\n\t"
+        "mov.b64 a, {%2, %3};\n\t"
+        "fma.rn.f32x2 d, a, %4, %5;\n\t"
+        "mov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "l"(b2), "l"(c2));
+}
+
+// acc += (a0, a1), packed fp32 add.
+__device__ __forceinline__ void fadd2_acc(uint64_t& acc, float a0, float a1) {
+    asm("{\n\t.reg .b64 a;\n\t"
+        "mov.b64 a, {%1, %2};\n\t"
+        "add.rn.f32x2 %0, %0, a;\n\t}"
+        : "+l"(acc)
+        : "f"(a0), "f"(a1));
 }
 
 // Two floats -> packed bf16x2 (round to nearest even); `lo` in bits [0, 16).
