@@ -93,6 +93,23 @@ def test_parity_other_scales():
         compare_all_rows(q, k, v, scale, FULL, 0, f"scale {scale}")
 
 
+@pytest.mark.parametrize("mask,chunk", [(FULL, 0), (BC, 500)])
+def test_running_max_jumps_force_rescaling(mask, chunk):
+    """Later key tiles carry much larger logits, so the running row max grows
+    far past the lazy-rescale threshold mid-sequence (and once more inside a
+    tile that is only partly allowed)."""
+    B, H, S, D = 1, 2, 1000, 128
+    q, k, v = wl.draw_qkv(B, H, S, S, D, seed=21, recipe="rms_qk")
+    k = k.float()
+    k[:, 300:428] *= 6.0   # keys across the tile 2/3 boundary: row max ~4 -> ~21 (log2 units)
+    k[:, 700:760] *= 12.0  # inside tile 5: row max -> ~40
+    compare_all_rows(q, k.to(torch.bfloat16), v, 1 / math.sqrt(D), mask, chunk, f"rescale m{mask}")
+    # descending: the largest logits come first, later tiles never rescale
+    k2 = wl.draw_qkv(B, H, S, S, D, seed=22, recipe="rms_qk")[1].float()
+    k2[:, :128] *= 10.0
+    compare_all_rows(q, k2.to(torch.bfloat16), v, 1 / math.sqrt(D), mask, chunk, f"no-rescale m{mask}")
+
+
 def test_constant_values_and_zero_queries():
     B, H, S, D = 1, 2, 700, 128
     q, k, _ = wl.draw_qkv(B, H, S, S, D, seed=11, recipe="rms_qk")

@@ -374,6 +374,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             kv_lim = static_cast<int>(min(static_cast<long long>(p.Skv), lim));
         }
         const float scale_log2 = p.scale_log2;
+        const uint64_t scale2 = pack_f32x2(scale_log2, scale_log2);
         float m = -INFINITY;  // reference max (log2 units) the exponentials are taken against
         float l = 0.0f;       // running row sum at that reference
         bool ok = true;
@@ -396,64 +397,86 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     for (int i = 0; i < 32; ++i)
                         if (c * 32 + i >= lim) s[c][i] = __float_as_uint(-INFINITY);
             }
-            // row max: eight independent 3-input max chains, then combine
-            float mxc[8];
+            // Row max over the tile: eight independent 3-input max chains.
+            auto tile_max = [&]() {
+                float mxc[8];
 #pragma unroll
-            for (int g = 0; g < 8; ++g) {
-                const uint32_t* v = &s[g >> 1][(g & 1) * 16];
-                float a = fmaxf(__uint_as_float(v[0]), __uint_as_float(v[1]));
+                for (int g = 0; g < 8; ++g) {
+                    const uint32_t* v = &s[g >> 1][(g & 1) * 16];
+                    float a = fmaxf(__uint_as_float(v[0]), __uint_as_float(v[1]));
 #pragma unroll
-                for (int i = 2; i < 16; i += 2) a = fmax3(a, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
-                mxc[g] = a;
-            }
-            const float mx = fmax3(fmax3(mxc[0], mxc[1], mxc[2]), fmax3(mxc[3], mxc[4], mxc[5]),
-                                   fmaxf(mxc[6], mxc[7]));
-            const float m_tile = mx * scale_log2;
-
-            float alpha = 1.0f;
-            bool rescale = false;
+                    for (int i = 2; i < 16; i += 2) a = fmax3(a, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+                    mxc[g] = a;
+                }
+                return fmax3(fmax3(mxc[0], mxc[1], mxc[2]), fmax3(mxc[3], mxc[4], mxc[5]), fmaxf(mxc[6], mxc[7]));
+            };
+            uint64_t lsum[4] = {0, 0, 0, 0};
+            uint32_t pa[2][16];  // packed P of keys 0-63, held until the reference max is settled
             if (j == 0) {
-                m = m_tile;
-            } else if (m_tile > m + kRescaleThreshold) {
-                alpha = ex2_approx(m - m_tile);
-                m = m_tile;
-                l *= alpha;
-                rescale = true;
-            }
-            if (__any_sync(0xffffffffu, rescale)) {
-                // O_t holds sum_k P_k V_k at the old reference: bring it to the
-                // new one before any half of this tile's P is released.
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(tO + uint32_t(c) * 32u, o);
-                    tmem_ld_wait(o);
+                // first tile: the reference max is the tile max
+                m = tile_max() * scale_log2;
+                const float m_use = (m == -INFINITY) ? 0.0f : m;
+                const uint64_t negm2 = pack_f32x2(-m_use, -m_use);
+                exp_chunk(s[0], scale2, negm2, pa[0], lsum);
+                exp_chunk(s[1], scale2, negm2, pa[1], lsum);
+            } else {
+                // Exponentiate keys 0-63 against the current reference while the
+                // tile max is computed alongside; only if the max grew past the
+                // threshold (rare) are O and l rescaled and keys 0-63 redone.
+                const float m_use0 = (m == -INFINITY) ? 0.0f : m;
+                const uint64_t negm2 = pack_f32x2(-m_use0, -m_use0);
+                exp_chunk(s[0], scale2, negm2, pa[0], lsum);
+                exp_chunk(s[1], scale2, negm2, pa[1], lsum);
+                const float m_tile = tile_max() * scale_log2;
+                const bool rescale = m_tile > m + kRescaleThreshold;
+                if (__any_sync(0xffffffffu, rescale)) {
+                    float alpha = 1.0f;
+                    if (rescale) {
+                        alpha = ex2_approx(m - m_tile);
+                        m = m_tile;
+                        l *= alpha;
+                        // redo keys 0-63 against the new reference
+                        const float m_use1 = m;
+                        const uint64_t negm2b = pack_f32x2(-m_use1, -m_use1);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    tmem_st32(tO + uint32_t(c) * 32u, o);
+                        for (int q = 0; q < 4; ++q) lsum[q] = 0;
+                        exp_chunk(s[0], scale2, negm2b, pa[0], lsum);
+                        exp_chunk(s[1], scale2, negm2b, pa[1], lsum);
+                    }
+                    // O_t holds sum_k P_k V_k at the old reference: bring it to
+                    // the new one before any of this tile's P is released.
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + uint32_t(c) * 32u, o);
+                        tmem_ld_wait(o);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st32(tO + uint32_t(c) * 32u, o);
+                    }
                 }
             }
-            const float m_use = (m == -INFINITY) ? 0.0f : m;
-            // P = exp2(S * scale*log2e - m) in two 64-key halves; each half goes
-            // to TMEM (over S columns already read) and is released to the MMA
-            // issuer on its own barrier.
-            const uint64_t scale2 = pack_f32x2(scale_log2, scale_log2);
-            const uint64_t negm2 = pack_f32x2(-m_use, -m_use);
-            uint64_t lsum[4] = {0, 0, 0, 0};
+            // release keys 0-63, then exponentiate and release keys 64-127
+            tmem_st16(tS, pa[0]);
+            tmem_st16(tS + 16u, pa[1]);
+            tmem_st_wait();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&bars->p_full[t][0]));
+            {
+                const float m_use = (m == -INFINITY) ? 0.0f : m;
+                const uint64_t negm2 = pack_f32x2(-m_use, -m_use);
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int c = hf * 2 + cc;
+                for (int c = 2; c < 4; ++c) {
                     uint32_t pk[16];
                     exp_chunk(s[c], scale2, negm2, pk, lsum);
                     tmem_st16(tS + uint32_t(c) * 16u, pk);
                 }
-                tmem_st_wait();
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(&bars->p_full[t][hf]));
             }
+            tmem_st_wait();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&bars->p_full[t][1]));
             {
                 float part = 0.0f;
 #pragma unroll
