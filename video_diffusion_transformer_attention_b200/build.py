@@ -51,15 +51,16 @@ def check_launch_registers(ptxas_log: str) -> int:
     """The forward kernel re-splits its registers with setmaxnreg, which is only
     safe if ptxas allocated exactly kLaunchRegs a thread at launch; a smaller
     allocation would leave setmaxnreg.inc waiting forever.  Returns the count."""
-    m = re.search(r"Compiling entry function '\w*attn_fwd_sm100_kernel\w*'.*?Used (\d+) registers",
-                  ptxas_log, flags=re.S)
-    if m is None:
+    found = re.findall(r"Compiling entry function '(\w*attn_fwd_sm100_kernel\w*)'.*?Used (\d+) registers",
+                       ptxas_log, flags=re.S)
+    if not found:
         raise RuntimeError("could not find the forward kernel's register count in the ptxas output")
-    used, expected = int(m.group(1)), _launch_regs_expected()
-    if used != expected:
-        raise RuntimeError(f"attn_fwd_sm100_kernel allocates {used} registers a thread, "
-                           f"the setmaxnreg split assumes {expected}")
-    return used
+    expected = _launch_regs_expected()
+    for name, used in found:
+        if int(used) != expected:
+            raise RuntimeError(f"{name} allocates {used} registers a thread, "
+                               f"the setmaxnreg split assumes {expected}")
+    return expected
 
 
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
