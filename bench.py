@@ -18,6 +18,7 @@ of the same workload (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -50,6 +51,27 @@ def load_peaks():
             p = json.load(f)
         return p, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("attn_fwd_sm100.cuh", "sm100_ptx.cuh"):
+        with open(os.path.join(ROOT, "video_diffusion_transformer_attention_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic():
+    """Per-launch DRAM bytes of the self-attention launch from the committed ncu
+    record, or None when the kernel source has changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "attn_fwd_sm100_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("kernel_source_sha256") != kernel_source_hash():
+        return None
+    return float(rec["traffic_per_launch_scaled"])
 
 
 def workload_config(name):
@@ -87,7 +109,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -329,7 +351,8 @@ def run_vdit(args):
             "config": {"workload": f"{args.workload} ({desc})", "l2": "inputs larger than L2 (3.1 GB per step)",
                        "parallelism": f"independent replicas x{world} (no collective)"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_sustained, "unit": "TFLOP/s",
-                         "frac": achieved / peak_sustained, "traffic": None,
+                         "frac": achieved / peak_sustained,
+                         "traffic": recorded_traffic() if args.workload == WORKLOAD else None,
                          "kernel": "attn_fwd_sm100_kernel (self-attention launch)",
                          "peak_kind": f"{peak_src} sustained bf16 (cuBLAS, power-capped)",
                          "frac_of_burst": achieved / peak_burst,
@@ -362,7 +385,7 @@ def main():
     ap.add_argument("--impl", choices=("vdit", "reference"), default="vdit")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(wl.WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=3)
-    ap.add_argument("--reference-seconds", type=float, default=20.0)
+    ap.add_argument("--reference-seconds", type=float, default=40.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "vdit":

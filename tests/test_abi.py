@@ -9,7 +9,7 @@ import pytest
 from video_diffusion_transformer_attention_b200 import binding as vb
 from video_diffusion_transformer_attention_b200.build import build
 
-HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "vdit_attn.h")
+INCLUDE = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -19,9 +19,12 @@ def built_library():
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(vdit_\w+)\s*\(", text)))
+    names = set()
+    for f in sorted(os.listdir(INCLUDE)):
+        if f.endswith(".h"):
+            text = re.sub(r"/\*.*?\*/", "", open(os.path.join(INCLUDE, f)).read(), flags=re.S)
+            names.update(re.findall(r"\b(vdit_\w+)\s*\(", text))
+    return sorted(names)
 
 
 def test_header_and_binding_agree():
@@ -87,6 +90,13 @@ def test_fwd_rejects_bad_arguments_before_any_launch(kw, status):
                           args["Sq"], args["Skv"], args["D"], args["scale"], args["mask_kind"],
                           args["chunk_tokens"], stream=0, check=False)
     assert st == status
+
+
+def test_testing_entry_point_rejects_bad_fault_or_limit():
+    args = (A, A * 3, A * 5, A * 7, A * 9, 1, 2, 64, 64, 128, 0.1, 0, 0)
+    assert vb.vdit_testing_attn_fwd(*args, 7, 10 ** 8, stream=0) == vb.VDIT_ERR_INVALID_ARG
+    assert vb.vdit_testing_attn_fwd(*args, vb.VDIT_TESTING_WITHHOLD_KV, 10, stream=0) == vb.VDIT_ERR_INVALID_ARG
+    assert vb.vdit_testing_attn_fwd(*args, vb.VDIT_TESTING_WITHHOLD_KV, 10 ** 11, stream=0) == vb.VDIT_ERR_INVALID_ARG
 
 
 def test_empty_call_is_a_no_op():

@@ -1,4 +1,4 @@
-"""ctypes binding of libvdit_attn.so: the C ABI of include/vdit_attn.h, same names.
+"""ctypes binding of libvdit_attn.so: the C ABI of include/*.h, same names.
 
 Argument marshalling only -- every step of the attention runs in the CUDA
 library.  Functions accept raw integers (device addresses, a cudaStream_t
@@ -27,7 +27,10 @@ VDIT_ERR_CUDA = 4
 VDIT_ERR_TIMEOUT = 5
 VDIT_ERR_WORKSPACE = 6
 
-# every entry point of include/vdit_attn.h
+VDIT_TESTING_NO_FAULT = 0
+VDIT_TESTING_WITHHOLD_KV = 1
+
+# every entry point declared in include/*.h
 EXPORTS = (
     "vdit_attn_plan",
     "vdit_attn_fwd",
@@ -35,6 +38,7 @@ EXPORTS = (
     "vdit_get_device_status",
     "vdit_status_string",
     "vdit_abi_version",
+    "vdit_testing_attn_fwd",
 )
 
 _lock = threading.Lock()
@@ -67,6 +71,8 @@ def lib() -> ctypes.CDLL:
             h.vdit_attn_fwd.argtypes = fwd_args + [vp]
             h.vdit_attn_fwd_ws.restype = c_int
             h.vdit_attn_fwd_ws.argtypes = fwd_args + [vp, c_size, vp]
+            h.vdit_testing_attn_fwd.restype = c_int
+            h.vdit_testing_attn_fwd.argtypes = fwd_args + [c_int, ctypes.c_ulonglong, vp]
             h.vdit_get_device_status.restype = c_int
             h.vdit_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
             h.vdit_status_string.restype = ctypes.c_char_p
@@ -132,6 +138,14 @@ def vdit_attn_fwd_ws(q, k, v, o, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_
     if check and st != VDIT_OK:
         raise VditError(st, "vdit_attn_fwd_ws")
     return st
+
+
+def vdit_testing_attn_fwd(q, k, v, o, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, fault,
+                          wait_timeout_ns, stream=None) -> int:
+    """Test-only forward with an injected fault (see include/vdit_attn_testing.h); returns the status."""
+    return int(lib().vdit_testing_attn_fwd(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), B, H, Sq, Skv, D,
+                                           float(scale), mask_kind, chunk_tokens, int(fault),
+                                           int(wait_timeout_ns), _stream(stream)))
 
 
 def vdit_get_device_status(stream=None):

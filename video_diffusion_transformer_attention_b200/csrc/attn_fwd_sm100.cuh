@@ -101,7 +101,12 @@ struct FwdParams {
     __nv_bfloat16* o;
     float* lse;
     unsigned long long timeout_ns;
+    int debug_flags;  // test-only fault injection (kDebug*); 0 in every product call
 };
+
+// Test-only: the producer withholds every K/V tile, so the MMA issuer's
+// bounded wait on the first K tile runs out and the timeout path runs.
+constexpr int kDebugWithholdKV = 1;
 
 // Written by kernels when a bounded wait runs out; read and cleared by the host.
 __device__ uint32_t g_status_word = 0;
@@ -276,7 +281,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 tma_load_4d(sQ + t * kTileBytes, &tm_q, bar, 0, h, q0 + t * kBlockM, b);
                 tma_load_4d(sQ + t * kTileBytes + kHalfBytes, &tm_q, bar, 64, h, q0 + t * kBlockM, b);
             }
-            for (int u = 0; u < 2 * n_kv; ++u) {
+            const int n_loads = (p.debug_flags & kDebugWithholdKV) ? 0 : 2 * n_kv;
+            for (int u = 0; u < n_loads; ++u) {
                 const int slot = u % kStages;
                 const uint32_t phase = uint32_t(u / kStages) & 1u;
                 if (!bounded_wait(smem_addr(&bars->kv_empty[slot]), phase ^ 1u, abort_flag, p.timeout_ns,

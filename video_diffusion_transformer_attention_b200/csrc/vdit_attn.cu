@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "vdit_attn.h"
+#include "vdit_attn_testing.h"
 #include "attn_fwd_sm100.cuh"
 
 namespace {
@@ -120,7 +121,7 @@ bool encode_bshd(CUtensorMap* map, const void* base, int B, int S, int H) {
 }
 
 vdit_status launch(const void* q, const void* k, const void* v, void* o, float* lse, const Shape& s, float scale,
-                   cudaStream_t stream) {
+                   int debug_flags, unsigned long long timeout_ns, cudaStream_t stream) {
     int dev = 0;
     vdit_status st = ensure_device(&dev);
     if (st != VDIT_OK) return st;
@@ -138,7 +139,8 @@ vdit_status launch(const void* q, const void* k, const void* v, void* o, float* 
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.o = static_cast<__nv_bfloat16*>(o);
     p.lse = lse;
-    p.timeout_ns = kDefaultWaitTimeoutNs;
+    p.timeout_ns = timeout_ns;
+    p.debug_flags = debug_flags;
     dim3 grid(grid_x(s.Sq), s.H, s.B);
     vdit::attn_fwd_sm100_kernel<<<grid, vdit::kNumThreads, vdit::kSmemBytes, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
@@ -146,7 +148,8 @@ vdit_status launch(const void* q, const void* k, const void* v, void* o, float* 
 
 vdit_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
                      int Skv, int D, float scale, int mask_kind, int chunk_tokens, void* workspace,
-                     size_t workspace_bytes, void* stream) {
+                     size_t workspace_bytes, void* stream, int debug_flags = 0,
+                     unsigned long long timeout_ns = kDefaultWaitTimeoutNs) {
     (void)workspace;
     (void)workspace_bytes;  // no shape needs a workspace in this version
     const Shape s{B, H, Sq, Skv, D, mask_kind, chunk_tokens};
@@ -167,7 +170,7 @@ vdit_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
             overlaps(lse, lse_bytes, k, kv_bytes) || overlaps(lse, lse_bytes, v, kv_bytes))
             return VDIT_ERR_INVALID_ARG;
     }
-    return launch(q, k, v, o, lse, s, scale, static_cast<cudaStream_t>(stream));
+    return launch(q, k, v, o, lse, s, scale, debug_flags, timeout_ns, static_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -222,6 +225,20 @@ vdit_status vdit_attn_fwd_ws(const void* q, const void* k, const void* v, void* 
     try {
         return fwd_impl(q, k, v, o, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, workspace,
                         workspace_bytes, stream);
+    } catch (...) {
+        return VDIT_ERR_CUDA;
+    }
+}
+
+vdit_status vdit_testing_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                                  int Sq, int Skv, int D, float scale, int mask_kind, int chunk_tokens,
+                                  int fault, unsigned long long wait_timeout_ns, void* stream) {
+    try {
+        if (fault != VDIT_TESTING_NO_FAULT && fault != VDIT_TESTING_WITHHOLD_KV) return VDIT_ERR_INVALID_ARG;
+        if (wait_timeout_ns < 1000000ull || wait_timeout_ns > 10000000000ull) return VDIT_ERR_INVALID_ARG;
+        const int flags = fault == VDIT_TESTING_WITHHOLD_KV ? vdit::kDebugWithholdKV : 0;
+        return fwd_impl(q, k, v, o, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, nullptr, 0, stream, flags,
+                        wait_timeout_ns);
     } catch (...) {
         return VDIT_ERR_CUDA;
     }
