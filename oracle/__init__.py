@@ -6,9 +6,11 @@ imports it, and it shares no code with the CUDA library.
 """
 from .oracle import (  # noqa: F401
     MASK_BLOCK_CAUSAL,
+    MASK_BLOCK_SPARSE,
     MASK_CROSS,
     MASK_FULL,
     attention,
     build,
     max_threads,
+    SPARSE_BLOCK,
 )

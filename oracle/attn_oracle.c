@@ -32,6 +32,12 @@
  *
  *   A(i) = { j : 0 <= j < Skv }                       FULL (0) and CROSS (2)
  *   A(i) = { j : j < Skv and floor(j/c) <= floor(i/c) } BLOCK_CAUSAL (1)
+ *   A(i) = { j : j < Skv and mask[b][h][i/128][j/128] }  BLOCK_SPARSE (3)
+ *
+ * BLOCK_SPARSE is the block-sparse attention of the sudonull.com page's
+ * optimisation list ("Sparse attention (VSA / Block Sparse): skips unimportant
+ * token pairs"): a caller-given byte per (128-query, 128-key) block says
+ * whether the pair of blocks attends.
  *
  * An empty A(i) gives O = 0 and LSE = -inf.  Subtracting M_i before exp is the
  * textbook overflow guard; it changes nothing in exact arithmetic.
@@ -50,6 +56,8 @@
 #define ORACLE_MASK_FULL 0
 #define ORACLE_MASK_BLOCK_CAUSAL 1
 #define ORACLE_MASK_CROSS 2
+#define ORACLE_MASK_BLOCK_SPARSE 3
+#define ORACLE_SPARSE_BLOCK 128
 
 /* bf16 is the upper half of an IEEE binary32; widening is exact. */
 static double widen_bf16(uint16_t bits) {
@@ -59,7 +67,9 @@ static double widen_bf16(uint16_t bits) {
     return (double)f;
 }
 
-/* Number of keys in A(i): the allowed set is always a prefix [0, n). */
+/* Keys j < n are candidates: the allowed set of FULL, CROSS and
+ * BLOCK_CAUSAL is exactly the prefix [0, n); BLOCK_SPARSE further needs the
+ * block bit (key_allowed). */
 static int64_t allowed_prefix(int mask_kind, int64_t i, int64_t Skv, int64_t chunk) {
     if (mask_kind == ORACLE_MASK_BLOCK_CAUSAL) {
         int64_t end = (i / chunk + 1) * chunk; /* first key of the next chunk */
@@ -68,31 +78,41 @@ static int64_t allowed_prefix(int mask_kind, int64_t i, int64_t Skv, int64_t chu
     return Skv;
 }
 
-/* One query row.  logits: scratch of Skv doubles. */
+static int key_allowed(int mask_kind, const uint8_t* mask_row, int64_t j) {
+    if (mask_kind != ORACLE_MASK_BLOCK_SPARSE) return 1;
+    return mask_row[j / ORACLE_SPARSE_BLOCK] != 0;
+}
+
+/* One query row.  logits: scratch of Skv doubles.  mask_row: the row's
+ * block-mask row (BLOCK_SPARSE only). */
 static void oracle_row(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                        int64_t H, int64_t Sq, int64_t Skv, int64_t D,
-                       double scale, int mask_kind, int64_t chunk,
+                       double scale, int mask_kind, int64_t chunk, const uint8_t* mask_row,
                        int64_t b, int64_t h, int64_t i,
                        double* logits, double* o_row, double* lse_out) {
     const uint16_t* qi = q + ((b * Sq + i) * H + h) * D;
     int64_t n = allowed_prefix(mask_kind, i, Skv, chunk);
     for (int64_t d = 0; d < D; ++d) o_row[d] = 0.0;
-    if (n <= 0) {
-        *lse_out = -INFINITY;
-        return;
-    }
-    /* l_ij = scale * <q_i, k_j> */
+    /* l_ij = scale * <q_i, k_j> for the allowed keys */
     double M = -INFINITY;
+    int64_t count = 0;
     for (int64_t j = 0; j < n; ++j) {
+        if (!key_allowed(mask_kind, mask_row, j)) continue;
         const uint16_t* kj = k + ((b * Skv + j) * H + h) * D;
         double dot = 0.0;
         for (int64_t d = 0; d < D; ++d) dot += widen_bf16(qi[d]) * widen_bf16(kj[d]);
         logits[j] = scale * dot;
         if (logits[j] > M) M = logits[j];
+        ++count;
+    }
+    if (count == 0) {
+        *lse_out = -INFINITY;
+        return;
     }
     /* Z_i and the unnormalised weighted sum of V rows */
     double Z = 0.0;
     for (int64_t j = 0; j < n; ++j) {
+        if (!key_allowed(mask_kind, mask_row, j)) continue;
         const uint16_t* vj = v + ((b * Skv + j) * H + h) * D;
         double w = exp(logits[j] - M);
         Z += w;
@@ -105,20 +125,25 @@ static void oracle_row(const uint16_t* q, const uint16_t* k, const uint16_t* v,
 /*
  * vdit_oracle_attn -- rows selected by `sel` (nsel triples b,h,i), or every row
  * in (b, h, i) order when sel == NULL (then nsel is ignored and B*H*Sq rows are
- * written).  o: [rows][D] doubles, lse: [rows] doubles.  nthreads <= 0 uses
- * the OpenMP default.  Returns 0, or -1 on a bad argument.
+ * written).  o: [rows][D] doubles, lse: [rows] doubles.  block_mask: for
+ * BLOCK_SPARSE, [B][H][ceil(Sq/128)][ceil(Skv/128)] bytes (nonzero = the
+ * blocks attend), else ignored.  nthreads <= 0 uses the OpenMP default.
+ * Returns 0, or -1 on a bad argument.
  */
 int vdit_oracle_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                      int64_t B, int64_t H, int64_t Sq, int64_t Skv, int64_t D,
-                     double scale, int mask_kind, int64_t chunk,
+                     double scale, int mask_kind, int64_t chunk, const uint8_t* block_mask,
                      const int64_t* sel, int64_t nsel,
                      double* o, double* lse, int nthreads) {
     if (!q || !k || !v || !o || !lse) return -1;
     if (B < 0 || H < 0 || Sq < 0 || Skv < 0 || D <= 0) return -1;
     if (mask_kind != ORACLE_MASK_FULL && mask_kind != ORACLE_MASK_BLOCK_CAUSAL &&
-        mask_kind != ORACLE_MASK_CROSS)
+        mask_kind != ORACLE_MASK_CROSS && mask_kind != ORACLE_MASK_BLOCK_SPARSE)
         return -1;
     if (mask_kind == ORACLE_MASK_BLOCK_CAUSAL && chunk <= 0) return -1;
+    if (mask_kind == ORACLE_MASK_BLOCK_SPARSE && !block_mask) return -1;
+    const int64_t nqb = (Sq + ORACLE_SPARSE_BLOCK - 1) / ORACLE_SPARSE_BLOCK;
+    const int64_t nkb = (Skv + ORACLE_SPARSE_BLOCK - 1) / ORACLE_SPARSE_BLOCK;
     int64_t rows = sel ? nsel : B * H * Sq;
     if (sel) {
         for (int64_t r = 0; r < rows; ++r) {
@@ -151,7 +176,11 @@ int vdit_oracle_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                     h = (r / Sq) % H;
                     i = r % Sq;
                 }
-                oracle_row(q, k, v, H, Sq, Skv, D, scale, mask_kind, chunk, b, h, i,
+                const uint8_t* mask_row =
+                    mask_kind == ORACLE_MASK_BLOCK_SPARSE
+                        ? block_mask + ((b * H + h) * nqb + i / ORACLE_SPARSE_BLOCK) * nkb
+                        : NULL;
+                oracle_row(q, k, v, H, Sq, Skv, D, scale, mask_kind, chunk, mask_row, b, h, i,
                            logits, o + r * D, lse + r);
             }
             free(logits);

@@ -21,6 +21,8 @@ import numpy as np
 MASK_FULL = 0
 MASK_BLOCK_CAUSAL = 1
 MASK_CROSS = 2
+MASK_BLOCK_SPARSE = 3
+SPARSE_BLOCK = 128
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "attn_oracle.c")
@@ -52,7 +54,7 @@ def _lib():
             h.vdit_oracle_attn.argtypes = [
                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                 ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
-                ctypes.c_double, ctypes.c_int, ctypes.c_int64,
+                ctypes.c_double, ctypes.c_int, ctypes.c_int64, ctypes.c_void_p,
                 ctypes.c_void_p, ctypes.c_int64,
                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
             ]
@@ -76,11 +78,13 @@ def _as_bits(x) -> np.ndarray:
 
 
 def attention(q_bits, k_bits, v_bits, scale: float, mask_kind: int = MASK_FULL,
-              chunk_tokens: int = 0, rows=None, threads: int = 0):
+              chunk_tokens: int = 0, rows=None, threads: int = 0, block_mask=None):
     """fp64 attention.
 
     q_bits: [B, Sq, H, D] uint16 (bf16 bits); k_bits, v_bits: [B, Skv, H, D].
     rows: None for every row, else an int array of shape [n, 3] of (b, h, i).
+    block_mask: for MASK_BLOCK_SPARSE, [B, H, ceil(Sq/128), ceil(Skv/128)]
+    (nonzero = the query block attends to the key block).
     Returns (O, LSE): O is [B, Sq, H, D] float64 (all rows) or [n, D];
     LSE is [B, H, Sq] float64 (all rows) or [n].
     """
@@ -99,9 +103,16 @@ def attention(q_bits, k_bits, v_bits, scale: float, mask_kind: int = MASK_FULL,
         n = sel.shape[0]
     o = np.zeros((n, D), dtype=np.float64)
     lse = np.zeros((n,), dtype=np.float64)
+    mask = None
+    if mask_kind == MASK_BLOCK_SPARSE:
+        nqb, nkb = -(-Sq // SPARSE_BLOCK), -(-Skv // SPARSE_BLOCK)
+        mask = np.ascontiguousarray(np.asarray(block_mask) != 0, dtype=np.uint8)
+        if mask.shape != (B, H, nqb, nkb):
+            raise ValueError(f"block_mask must be [B, H, {nqb}, {nkb}]")
     rc = _lib().vdit_oracle_attn(
         q.ctypes.data, k.ctypes.data, v.ctypes.data,
         B, H, Sq, Skv, D, float(scale), int(mask_kind), int(chunk_tokens),
+        None if mask is None else mask.ctypes.data,
         None if sel is None else sel.ctypes.data, n,
         o.ctypes.data, lse.ctypes.data, int(threads))
     if rc != 0:

@@ -239,3 +239,66 @@ def test_oracle_rejects_bad_arguments():
         attention(qb, qb, qb, 0.5, MASK_BLOCK_CAUSAL, 0)
     with pytest.raises(TypeError):
         attention(qb.astype(np.float32), qb, qb, 0.5)
+
+
+# ---------------------------------------------------------------- block-sparse
+
+from oracle import MASK_BLOCK_SPARSE, SPARSE_BLOCK  # noqa: E402
+
+
+def expand_block_mask(bm, Sq, Skv):
+    """[B,H,nqb,nkb] block mask -> [B,H,Sq,Skv] boolean token mask."""
+    t = torch.from_numpy(np.asarray(bm) != 0)
+    t = t.repeat_interleave(SPARSE_BLOCK, dim=2).repeat_interleave(SPARSE_BLOCK, dim=3)
+    return t[:, :, :Sq, :Skv]
+
+
+def test_block_sparse_all_ones_is_full():
+    rng = np.random.default_rng(40)
+    B, H, Sq, Skv, D = 1, 2, 300, 270, 16
+    qb, kb, vb = rand_bits(rng, (B, Sq, H, D)), rand_bits(rng, (B, Skv, H, D)), rand_bits(rng, (B, Skv, H, D))
+    ones = np.ones((B, H, 3, 3), np.uint8)
+    o, lse = attention(qb, kb, vb, 0.25, MASK_BLOCK_SPARSE, block_mask=ones)
+    o_f, l_f = attention(qb, kb, vb, 0.25, MASK_CROSS)
+    np.testing.assert_array_equal(o, o_f)
+    np.testing.assert_array_equal(lse, l_f)
+
+
+def test_block_sparse_block_causal_pattern_is_block_causal():
+    rng = np.random.default_rng(41)
+    B, H, S, D, c = 1, 2, 600, 16, 256  # chunks of two 128-token blocks
+    qb, kb, vb = (rand_bits(rng, (B, S, H, D)) for _ in range(3))
+    nb = -(-S // SPARSE_BLOCK)
+    qi = np.arange(nb)[:, None] * SPARSE_BLOCK // c
+    kj = np.arange(nb)[None, :] * SPARSE_BLOCK // c
+    bm = np.broadcast_to((kj <= qi).astype(np.uint8), (B, H, nb, nb))
+    o, lse = attention(qb, kb, vb, 0.3, MASK_BLOCK_SPARSE, block_mask=bm)
+    o_c, l_c = attention(qb, kb, vb, 0.3, MASK_BLOCK_CAUSAL, c)
+    np.testing.assert_array_equal(o, o_c)
+    np.testing.assert_array_equal(lse, l_c)
+
+
+def test_block_sparse_matches_torch_sdpa_with_the_expanded_mask():
+    rng = np.random.default_rng(42)
+    B, H, Sq, Skv, D = 2, 2, 400, 333, 16
+    qb, kb, vb = rand_bits(rng, (B, Sq, H, D)), rand_bits(rng, (B, Skv, H, D)), rand_bits(rng, (B, Skv, H, D))
+    bm = (rng.random((B, H, 4, 3)) < 0.5).astype(np.uint8)
+    bm[0, 0, 1, :] = 0  # one query block of one head attends to nothing
+    bm[1, 1, :, 2] = 1
+    o, lse = attention(qb, kb, vb, 0.25, MASK_BLOCK_SPARSE, block_mask=bm)
+    mask = expand_block_mask(bm, Sq, Skv)
+    has_key = mask.any(dim=-1).numpy()  # [B,H,Sq]
+    o_ref, l_ref = sdpa_reference(qb, kb, vb, 0.25, mask)
+    for b in range(B):
+        for h in range(H):
+            rows = has_key[b, h]
+            np.testing.assert_allclose(o[b, rows, h], o_ref[b, rows, h], rtol=0, atol=1e-12)
+            np.testing.assert_allclose(lse[b, h, rows], l_ref[b, h, rows], rtol=0, atol=1e-12)
+            assert np.all(o[b, ~rows, h] == 0.0) and np.all(np.isneginf(lse[b, h, ~rows]))
+    assert (~has_key).any()
+
+
+def test_block_sparse_rejects_a_wrong_mask_shape():
+    qb = np.zeros((1, 200, 1, 8), np.uint16)
+    with pytest.raises(ValueError):
+        attention(qb, qb, qb, 0.5, MASK_BLOCK_SPARSE, block_mask=np.ones((1, 1, 1, 1)))
