@@ -78,7 +78,9 @@ def workload_config(name):
     w = wl.WORKLOADS[name]
     desc = "; ".join(
         f"{c.name}: B={c.B} H={c.H} Sq={c.Sq} Skv={c.Skv} D={c.D} mask="
-        f"{['full', 'block_causal', 'cross'][c.mask_kind]}" + (f" chunk={c.chunk_tokens}" if c.chunk_tokens else "")
+        f"{['full', 'block_causal', 'cross', 'block_sparse'][c.mask_kind]}"
+        + (f" chunk={c.chunk_tokens}" if c.chunk_tokens else "")
+        + (f" density={wl.SPARSE_DENSITY}" if c.mask_kind == wl.MASK_BLOCK_SPARSE else "")
         for c in w.calls)
     return w, desc
 
@@ -154,15 +156,23 @@ def oracle_sample(inp, w, seconds_budget=20.0, seed=0):
         qb, kb, vb = wl.bf16_bits(q), wl.bf16_bits(k), wl.bf16_bits(v)
         # an equal share of the budget per call, at about 0.5 GFLOP/s per core
         # for this plain fp64 loop
-        flops_row = 4.0 * call.D * call.Skv
+        sparse = call.mask_kind == wl.MASK_BLOCK_SPARSE
+        flops_row = 4.0 * call.D * call.Skv * (wl.SPARSE_DENSITY if sparse else 1.0)
         n = int(max(8, min(call.B * call.H * call.Sq,
                           seconds_budget / len(w.calls) * 0.5e9 * oracle.max_threads() / flops_row)))
         rows = np.stack([rng.integers(0, call.B, n), rng.integers(0, call.H, n),
                          rng.integers(0, call.Sq, n)], axis=1)
+        mask = inp["block_mask"].numpy() if sparse else None
         t0 = time.perf_counter()
-        oracle.attention(qb, kb, vb, call.scale, call.mask_kind, call.chunk_tokens, rows=rows)
+        oracle.attention(qb, kb, vb, call.scale, call.mask_kind, call.chunk_tokens, rows=rows, block_mask=mask)
         dt = time.perf_counter() - t0
-        f = flops_row * n
+        if sparse:
+            # exact allowed keys of the sampled rows
+            blk = np.minimum(wl.SPARSE_BLOCK, call.Skv - wl.SPARSE_BLOCK * np.arange(mask.shape[-1]))
+            keys = (mask[rows[:, 0], rows[:, 1], rows[:, 2] // wl.SPARSE_BLOCK] != 0) @ blk
+            f = 4.0 * call.D * float(keys.sum())
+        else:
+            f = flops_row * n
         total_flops += f
         total_time += dt
         parts.append(f"{call.name}: {n} rows x {call.Skv} keys")
@@ -248,12 +258,17 @@ def run_vdit(args):
                      torch.empty((call.B, call.H, call.Sq), dtype=torch.float32, device=dev)))
     stream = torch.cuda.Stream(device=dev)
     sptr = int(stream.cuda_stream)
-    flops_per_call = [fl.attn_flops(c) for c in w.calls]
+    mask_cpu = inp_cpu.get("block_mask")
+    flops_per_call = [fl.attn_flops(c, mask_cpu) for c in w.calls]
     step_flops = sum(flops_per_call)
 
     def launch(i, call, q, k, v, o, lse):
-        vb.vdit_attn_fwd(q, k, v, o, lse, call.B, call.H, call.Sq, call.Skv, call.D, call.scale,
-                         call.mask_kind, call.chunk_tokens, sptr)
+        if call.mask_kind == wl.MASK_BLOCK_SPARSE:
+            vb.vdit_attn_fwd_block_sparse(q, k, v, o, lse, inp["block_mask"], call.B, call.H, call.Sq, call.Skv,
+                                          call.D, call.scale, sptr)
+        else:
+            vb.vdit_attn_fwd(q, k, v, o, lse, call.B, call.H, call.Sq, call.Skv, call.D, call.scale,
+                             call.mask_kind, call.chunk_tokens, sptr)
 
     def step(events=None):
         for i, call in enumerate(w.calls):

@@ -59,7 +59,12 @@ typedef enum {
     VDIT_MASK_BLOCK_CAUSAL = 1,
     /* Same arithmetic as FULL; the caller says the keys are a short text
      * sequence (Skv << Sq), e.g. 512 text tokens. */
-    VDIT_MASK_CROSS = 2
+    VDIT_MASK_CROSS = 2,
+    /* A(i) = { j : mask[b][h][i / 128][j / 128] != 0 }, a caller-given byte
+     * per (128-query, 128-key) block pair; key blocks no query of a tile pair
+     * attends to are skipped.  Only through vdit_attn_fwd_block_sparse (and
+     * vdit_attn_plan).  Skv <= 262,144. */
+    VDIT_MASK_BLOCK_SPARSE = 3
 } vdit_mask_kind;
 
 typedef enum {
@@ -96,7 +101,9 @@ vdit_status vdit_attn_plan(int B, int H, int Sq, int Skv, int D, int mask_kind,
  *   scale   : multiplies q.k before the softmax (1/sqrt(D) for the Wan
  *             configurations); finite and > 0.
  *   mask_kind, chunk_tokens : see vdit_mask_kind; chunk_tokens is ignored
- *             unless mask_kind == VDIT_MASK_BLOCK_CAUSAL.
+ *             unless mask_kind == VDIT_MASK_BLOCK_CAUSAL.  mask_kind
+ *             VDIT_MASK_BLOCK_SPARSE is rejected here (INVALID_ARG): it needs
+ *             vdit_attn_fwd_block_sparse.
  * B == 0, H == 0 or Sq == 0 is a valid empty call: VDIT_OK, nothing launched.
  * Returns VDIT_ERR_CUDA if the launch itself fails.  Timeouts inside the
  * kernel are reported later by vdit_get_device_status.
@@ -105,6 +112,24 @@ vdit_status vdit_attn_fwd(const void* q, const void* k, const void* v, void* o,
                           float* lse, int B, int H, int Sq, int Skv, int D,
                           float scale, int mask_kind, int chunk_tokens,
                           void* stream);
+
+/*
+ * vdit_attn_fwd_block_sparse -- block-sparse attention: the "Sparse attention
+ * (VSA / Block Sparse): skips unimportant token pairs" item of the
+ * optimisation list in "Realtime video generation: FLOPS calculation and
+ * optimizations" (sudonull.com).
+ *   block_mask : device bytes [B][H][ceil(Sq/128)][ceil(Skv/128)], row-major;
+ *                nonzero = query block i/128 attends to key block j/128.
+ *                Caller-owned, read-only, any alignment.
+ *   other arguments as vdit_attn_fwd.
+ * A query row whose blocks attend to no key gets O = 0 and LSE = -inf.
+ * VDIT_ERR_INVALID_ARG for a NULL mask or Skv > 262,144.
+ */
+vdit_status vdit_attn_fwd_block_sparse(const void* q, const void* k,
+                                       const void* v, void* o, float* lse,
+                                       const uint8_t* block_mask, int B, int H,
+                                       int Sq, int Skv, int D, float scale,
+                                       void* stream);
 
 /*
  * vdit_attn_fwd_ws -- vdit_attn_fwd with a caller-owned device workspace of

@@ -55,7 +55,8 @@ def test_plan_reports_grid_and_zero_workspace():
 @pytest.mark.parametrize("args,status", [
     ((1, 1, 16, 16, 64, 0, 0), vb.VDIT_ERR_UNSUPPORTED),
     ((1, 1, 16, 0, 128, 0, 0), vb.VDIT_ERR_INVALID_ARG),
-    ((1, 1, 16, 16, 128, 3, 0), vb.VDIT_ERR_INVALID_ARG),
+    ((1, 1, 16, 16, 128, 4, 0), vb.VDIT_ERR_INVALID_ARG),
+    ((1, 1, 16, 262145, 128, 3, 0), vb.VDIT_ERR_INVALID_ARG),
     ((1, 1, 16, 16, 128, 1, 0), vb.VDIT_ERR_INVALID_ARG),
     ((1, 1, 16, 32, 128, 1, 8), vb.VDIT_ERR_INVALID_ARG),
     ((-1, 1, 16, 16, 128, 0, 0), vb.VDIT_ERR_INVALID_ARG),
@@ -97,6 +98,20 @@ def test_testing_entry_point_rejects_bad_fault_or_limit():
     assert vb.vdit_testing_attn_fwd(*args, 7, 10 ** 8, stream=0) == vb.VDIT_ERR_INVALID_ARG
     assert vb.vdit_testing_attn_fwd(*args, vb.VDIT_TESTING_WITHHOLD_KV, 10, stream=0) == vb.VDIT_ERR_INVALID_ARG
     assert vb.vdit_testing_attn_fwd(*args, vb.VDIT_TESTING_WITHHOLD_KV, 10 ** 11, stream=0) == vb.VDIT_ERR_INVALID_ARG
+
+
+def test_block_sparse_needs_its_entry_point_and_a_mask():
+    assert vb.vdit_attn_plan(1, 2, 300, 262144, 128, vb.VDIT_MASK_BLOCK_SPARSE, 0)[1] == 4
+    args = (A, A * 3, A * 5, A * 7, A * 9)
+    # the plain forward does not take the block-sparse mask kind
+    assert vb.vdit_attn_fwd(*args, 1, 2, 64, 64, 128, 0.1, vb.VDIT_MASK_BLOCK_SPARSE, 0, stream=0,
+                            check=False) == vb.VDIT_ERR_INVALID_ARG
+    assert vb.vdit_attn_fwd_block_sparse(*args, None, 1, 2, 64, 64, 128, 0.1, stream=0,
+                                         check=False) == vb.VDIT_ERR_INVALID_ARG
+    assert vb.vdit_attn_fwd_block_sparse(*args, A * 11, 1, 2, 64, 300000, 128, 0.1, stream=0,
+                                         check=False) == vb.VDIT_ERR_INVALID_ARG
+    assert vb.vdit_attn_fwd_block_sparse(*args, A * 11, 1, 2, 64, 64, 96, 0.1, stream=0,
+                                         check=False) == vb.VDIT_ERR_UNSUPPORTED
 
 
 def test_empty_call_is_a_no_op():

@@ -18,6 +18,8 @@ LIB_PATH = os.path.join(HERE, "libvdit_attn.so")
 VDIT_MASK_FULL = 0
 VDIT_MASK_BLOCK_CAUSAL = 1
 VDIT_MASK_CROSS = 2
+VDIT_MASK_BLOCK_SPARSE = 3
+SPARSE_BLOCK = 128
 
 VDIT_OK = 0
 VDIT_ERR_INVALID_ARG = 1
@@ -35,6 +37,7 @@ EXPORTS = (
     "vdit_attn_plan",
     "vdit_attn_fwd",
     "vdit_attn_fwd_ws",
+    "vdit_attn_fwd_block_sparse",
     "vdit_get_device_status",
     "vdit_status_string",
     "vdit_abi_version",
@@ -71,6 +74,9 @@ def lib() -> ctypes.CDLL:
             h.vdit_attn_fwd.argtypes = fwd_args + [vp]
             h.vdit_attn_fwd_ws.restype = c_int
             h.vdit_attn_fwd_ws.argtypes = fwd_args + [vp, c_size, vp]
+            h.vdit_attn_fwd_block_sparse.restype = c_int
+            h.vdit_attn_fwd_block_sparse.argtypes = [vp, vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int,
+                                                     c_float, vp]
             h.vdit_testing_attn_fwd.restype = c_int
             h.vdit_testing_attn_fwd.argtypes = fwd_args + [c_int, ctypes.c_ulonglong, vp]
             h.vdit_get_device_status.restype = c_int
@@ -140,6 +146,16 @@ def vdit_attn_fwd_ws(q, k, v, o, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_
     return st
 
 
+def vdit_attn_fwd_block_sparse(q, k, v, o, lse, block_mask, B, H, Sq, Skv, D, scale, stream=None,
+                               check=True) -> int:
+    """Block-sparse forward; block_mask is a device uint8 [B, H, ceil(Sq/128), ceil(Skv/128)]."""
+    st = lib().vdit_attn_fwd_block_sparse(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), _addr(block_mask),
+                                          B, H, Sq, Skv, D, float(scale), _stream(stream))
+    if check and st != VDIT_OK:
+        raise VditError(st, "vdit_attn_fwd_block_sparse")
+    return st
+
+
 def vdit_testing_attn_fwd(q, k, v, o, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, fault,
                           wait_timeout_ns, stream=None) -> int:
     """Test-only forward with an injected fault (see include/vdit_attn_testing.h); returns the status."""
@@ -176,3 +192,23 @@ def attention(q, k, v, scale=None, mask_kind=VDIT_MASK_FULL, chunk_tokens=0, out
             raise ValueError("q, k, v, out must be contiguous CUDA bf16 tensors")
     vdit_attn_fwd(q, k, v, out, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, stream)
     return (out, lse) if return_lse else out
+
+
+def attention_block_sparse(q, k, v, block_mask, scale=None, out=None, lse=None, stream=None):
+    """Convenience wrapper over vdit_attn_fwd_block_sparse (CUDA bf16 [B, S, H, D] tensors,
+    block_mask a CUDA uint8 tensor [B, H, ceil(Sq/128), ceil(Skv/128)]).  Returns (o, lse)."""
+    import torch
+    B, Sq, H, D = q.shape
+    Skv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / float(D) ** 0.5
+    nqb, nkb = -(-Sq // SPARSE_BLOCK), -(-Skv // SPARSE_BLOCK)
+    if block_mask.dtype != torch.uint8 or tuple(block_mask.shape) != (B, H, nqb, nkb) or not block_mask.is_cuda \
+            or not block_mask.is_contiguous():
+        raise ValueError(f"block_mask must be a contiguous CUDA uint8 tensor [B, H, {nqb}, {nkb}]")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    vdit_attn_fwd_block_sparse(q, k, v, out, lse, block_mask, B, H, Sq, Skv, D, scale, stream)
+    return out, lse

@@ -69,6 +69,11 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when th
 constexpr int kMaskFull = 0;
 constexpr int kMaskBlockCausal = 1;
 constexpr int kMaskCross = 2;
+constexpr int kMaskBlockSparse = 3;
+constexpr int kSparseBlock = 128;        // block-mask granularity = the 128-row/128-key tiles
+constexpr int kMaxSparseKvBlocks = 2048; // key blocks a block-sparse call may have (Skv <= 262,144)
+constexpr uint16_t kListKvMask = 0x3FFF; // list entry: key block | allowed for tile 0 << 14 | tile 1 << 15
+constexpr int kListWarp = 10;
 
 // Device status word codes (OR-ed together).
 constexpr uint32_t kStatusTimeout = 1u;
@@ -91,7 +96,8 @@ struct __align__(8) Barriers {
 constexpr int kSmemQ = 0;
 constexpr int kSmemKV = kQTiles * kTileBytes;
 constexpr int kSmemBar = kSmemKV + kStages * kTileBytes;
-constexpr int kSmemBytes = kSmemBar + int(sizeof(Barriers)) + 1024;  // + alignment slack
+constexpr int kSmemList = kSmemBar + ((int(sizeof(Barriers)) + 15) / 16) * 16;  // block-sparse tile list
+constexpr int kSmemBytes = kSmemList + kMaxSparseKvBlocks * 2 + 16 + 1024;     // + alignment slack
 
 struct FwdParams {
     int B, H, Sq, Skv;
@@ -102,6 +108,8 @@ struct FwdParams {
     float* lse;
     unsigned long long timeout_ns;
     int debug_flags;  // test-only fault injection (kDebug*); 0 in every product call
+    const uint8_t* block_mask;  // block-sparse: [B][H][n_qb][n_kvb], nonzero = attend
+    int n_qb, n_kvb;            // ceil(Sq / 128), ceil(Skv / 128)
 };
 
 // Test-only: the producer withholds every K/V tile, so the MMA issuer's
@@ -253,10 +261,32 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         tmem_alloc(smem_addr(&bars->tmem_base), kTmemCols);
         tmem_relinquish();
     }
+    uint16_t* kv_list = reinterpret_cast<uint16_t*>(smem + kSmemList);
+    int* kv_list_len = reinterpret_cast<int*>(smem + kSmemList + kMaxSparseKvBlocks * 2);
+    if (p.mask_kind == kMaskBlockSparse && warp == kListWarp) {
+        // Compact the key blocks either query tile of this CTA attends to,
+        // in ascending order, each tagged with which of the two tiles may use it.
+        const int qb0 = q0 / kSparseBlock;
+        const uint8_t* row0 = p.block_mask + ((static_cast<size_t>(b) * p.H + h) * p.n_qb + qb0) * p.n_kvb;
+        const bool has_row1 = qb0 + 1 < p.n_qb;
+        int count = 0;
+        for (int base = 0; base < p.n_kvb; base += 32) {
+            const int kv = base + lane;
+            const bool a0 = kv < p.n_kvb && row0[kv] != 0;
+            const bool a1 = has_row1 && kv < p.n_kvb && row0[p.n_kvb + kv] != 0;
+            const uint32_t ballot = __ballot_sync(0xffffffffu, a0 || a1);
+            if (a0 || a1)
+                kv_list[count + __popc(ballot & ((1u << lane) - 1u))] =
+                    uint16_t(kv | (a0 ? 1 << 14 : 0) | (a1 ? 1 << 15 : 0));
+            count += __popc(ballot);
+        }
+        if (lane == 0) *kv_list_len = count;
+    }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = bars->tmem_base;
+    const bool sparse = p.mask_kind == kMaskBlockSparse;
 
     // Keys this CTA needs: all of them, or for block-causal everything up to
     // the end of the chunk that holds the CTA's last valid query row.
@@ -266,7 +296,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const long long lim = (static_cast<long long>(last_row / p.chunk) + 1) * p.chunk;
         kv_end = static_cast<int>(min(static_cast<long long>(p.Skv), lim));
     }
-    const int n_kv = (kv_end + kBlockN - 1) / kBlockN;
+    const int n_kv = sparse ? *kv_list_len : (kv_end + kBlockN - 1) / kBlockN;
 
     const uint32_t sQ = smem_addr(smem + kSmemQ);
     const uint32_t sKV = smem_addr(smem + kSmemKV);
@@ -275,7 +305,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         setmaxnreg_dec<kControlRegs>();
         if (warp == kLoadWarp && lane == 0) {
             // ------------------------------------------------ TMA producer
-            for (int t = 0; t < kQTiles; ++t) {
+            for (int t = 0; n_kv > 0 && t < kQTiles; ++t) {
                 const uint32_t bar = smem_addr(&bars->q_full[t]);
                 mbar_arrive_expect_tx(bar, kTileBytes);
                 tma_load_4d(sQ + t * kTileBytes, &tm_q, bar, 0, h, q0 + t * kBlockM, b);
@@ -290,7 +320,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     break;
                 const uint32_t full = smem_addr(&bars->kv_full[slot]);
                 const CUtensorMap* map = (u & 1) ? &tm_v : &tm_k;
-                const int row = (u >> 1) * kBlockN;
+                const int row = (sparse ? int(kv_list[u >> 1] & kListKvMask) : (u >> 1)) * kBlockN;
                 mbar_arrive_expect_tx(full, kTileBytes);
                 tma_load_4d(sKV + slot * kTileBytes, map, full, 0, h, row, b);
                 tma_load_4d(sKV + slot * kTileBytes + kHalfBytes, map, full, 64, h, row, b);
@@ -304,7 +334,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             const uint64_t k_desc0 = smem_desc_sw128(sKV, 16, 1024);
             const uint64_t v_desc0 = smem_desc_sw128(sKV, kHalfBytes, 1024);
             constexpr uint64_t kSlotStep = kTileBytes >> 4;
-            bool ok = bounded_wait(smem_addr(&bars->q_full[0]), 0, abort_flag, p.timeout_ns, kSiteMma) &&
+            bool ok = n_kv > 0 &&
+                      bounded_wait(smem_addr(&bars->q_full[0]), 0, abort_flag, p.timeout_ns, kSiteMma) &&
                       bounded_wait(smem_addr(&bars->q_full[1]), 0, abort_flag, p.timeout_ns, kSiteMma);
             // prologue: S_0 and S_1 against K_0
             if (ok) ok = bounded_wait(smem_addr(&bars->kv_full[0]), 0, abort_flag, p.timeout_ns, kSiteMma);
@@ -395,7 +426,14 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c) tmem_ld_wait(s[c]);
 
-            const int lim = kv_lim - j * kBlockN;
+            // keys of this tile allowed for the row: [0, lim) of the tile
+            int lim;
+            if (sparse) {
+                const uint32_t e = kv_list[j];
+                lim = ((e >> (14 + t)) & 1u) ? p.Skv - int(e & kListKvMask) * kBlockN : 0;
+            } else {
+                lim = kv_lim - j * kBlockN;
+            }
             if (lim < kBlockN) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
@@ -492,7 +530,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             }
         }
 
-        if (ok) ok = warp_wait(smem_addr(&bars->o_full[t]), 0, abort_flag, p.timeout_ns, kSiteSoftmax);
+        // With no key tile at all (an empty block-sparse list) O stays 0 and
+        // LSE = -inf; nothing was issued, so there is nothing to wait for.
+        if (ok && n_kv > 0) ok = warp_wait(smem_addr(&bars->o_full[t]), 0, abort_flag, p.timeout_ns, kSiteSoftmax);
         if (ok) {
             tc_fence_after_sync();
             const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
@@ -500,8 +540,13 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t o[32];
-                tmem_ld32(tO + uint32_t(c) * 32u, o);
-                tmem_ld_wait(o);
+                if (n_kv > 0) {
+                    tmem_ld32(tO + uint32_t(c) * 32u, o);
+                    tmem_ld_wait(o);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = 0u;
+                }
                 uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i)

@@ -29,7 +29,11 @@ struct Shape {
 
 vdit_status check_shape(const Shape& s, bool check_scale, float scale) {
     if (s.B < 0 || s.H < 0 || s.Sq < 0 || s.Skv < 1 || s.D < 1) return VDIT_ERR_INVALID_ARG;
-    if (s.mask_kind != VDIT_MASK_FULL && s.mask_kind != VDIT_MASK_BLOCK_CAUSAL && s.mask_kind != VDIT_MASK_CROSS)
+    if (s.mask_kind != VDIT_MASK_FULL && s.mask_kind != VDIT_MASK_BLOCK_CAUSAL && s.mask_kind != VDIT_MASK_CROSS &&
+        s.mask_kind != VDIT_MASK_BLOCK_SPARSE)
+        return VDIT_ERR_INVALID_ARG;
+    if (s.mask_kind == VDIT_MASK_BLOCK_SPARSE &&
+        (s.Skv + vdit::kSparseBlock - 1) / vdit::kSparseBlock > vdit::kMaxSparseKvBlocks)
         return VDIT_ERR_INVALID_ARG;
     if (s.D != vdit::kHeadDim) return VDIT_ERR_UNSUPPORTED;
     if (s.mask_kind == VDIT_MASK_BLOCK_CAUSAL && (s.chunk < 1 || s.Sq != s.Skv)) return VDIT_ERR_INVALID_ARG;
@@ -120,8 +124,9 @@ bool encode_bshd(CUtensorMap* map, const void* base, int B, int S, int H) {
     return r == CUDA_SUCCESS;
 }
 
-vdit_status launch(const void* q, const void* k, const void* v, void* o, float* lse, const Shape& s, float scale,
-                   int debug_flags, unsigned long long timeout_ns, cudaStream_t stream) {
+vdit_status launch(const void* q, const void* k, const void* v, void* o, float* lse, const uint8_t* block_mask,
+                   const Shape& s, float scale, int debug_flags, unsigned long long timeout_ns,
+                   cudaStream_t stream) {
     int dev = 0;
     vdit_status st = ensure_device(&dev);
     if (st != VDIT_OK) return st;
@@ -141,6 +146,9 @@ vdit_status launch(const void* q, const void* k, const void* v, void* o, float* 
     p.lse = lse;
     p.timeout_ns = timeout_ns;
     p.debug_flags = debug_flags;
+    p.block_mask = block_mask;
+    p.n_qb = (s.Sq + vdit::kSparseBlock - 1) / vdit::kSparseBlock;
+    p.n_kvb = (s.Skv + vdit::kSparseBlock - 1) / vdit::kSparseBlock;
     dim3 grid(grid_x(s.Sq), s.H, s.B);
     vdit::attn_fwd_sm100_kernel<<<grid, vdit::kNumThreads, vdit::kSmemBytes, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
@@ -149,13 +157,15 @@ vdit_status launch(const void* q, const void* k, const void* v, void* o, float* 
 vdit_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
                      int Skv, int D, float scale, int mask_kind, int chunk_tokens, void* workspace,
                      size_t workspace_bytes, void* stream, int debug_flags = 0,
-                     unsigned long long timeout_ns = kDefaultWaitTimeoutNs) {
+                     unsigned long long timeout_ns = kDefaultWaitTimeoutNs,
+                     const uint8_t* block_mask = nullptr) {
     (void)workspace;
     (void)workspace_bytes;  // no shape needs a workspace in this version
     const Shape s{B, H, Sq, Skv, D, mask_kind, chunk_tokens};
     vdit_status st = check_shape(s, true, scale);
     if (st != VDIT_OK) return st;
     if (B == 0 || H == 0 || Sq == 0) return VDIT_OK;
+    if ((mask_kind == VDIT_MASK_BLOCK_SPARSE) != (block_mask != nullptr)) return VDIT_ERR_INVALID_ARG;
     if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return VDIT_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return VDIT_ERR_MISALIGNED;
@@ -170,7 +180,15 @@ vdit_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
             overlaps(lse, lse_bytes, k, kv_bytes) || overlaps(lse, lse_bytes, v, kv_bytes))
             return VDIT_ERR_INVALID_ARG;
     }
-    return launch(q, k, v, o, lse, s, scale, debug_flags, timeout_ns, static_cast<cudaStream_t>(stream));
+    if (block_mask != nullptr) {
+        const size_t mask_bytes = size_t(B) * size_t(H) * size_t((Sq + vdit::kSparseBlock - 1) / vdit::kSparseBlock) *
+                                  size_t((Skv + vdit::kSparseBlock - 1) / vdit::kSparseBlock);
+        if (overlaps(block_mask, mask_bytes, o, q_bytes) ||
+            (lse != nullptr && overlaps(block_mask, mask_bytes, lse, size_t(B) * size_t(H) * size_t(Sq) * 4)))
+            return VDIT_ERR_INVALID_ARG;
+    }
+    return launch(q, k, v, o, lse, block_mask, s, scale, debug_flags, timeout_ns,
+                  static_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -225,6 +243,18 @@ vdit_status vdit_attn_fwd_ws(const void* q, const void* k, const void* v, void* 
     try {
         return fwd_impl(q, k, v, o, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, workspace,
                         workspace_bytes, stream);
+    } catch (...) {
+        return VDIT_ERR_CUDA;
+    }
+}
+
+vdit_status vdit_attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                                       const uint8_t* block_mask, int B, int H, int Sq, int Skv, int D, float scale,
+                                       void* stream) {
+    try {
+        if (B > 0 && H > 0 && Sq > 0 && block_mask == nullptr) return VDIT_ERR_INVALID_ARG;
+        return fwd_impl(q, k, v, o, lse, B, H, Sq, Skv, D, scale, VDIT_MASK_BLOCK_SPARSE, 0, nullptr, 0, stream, 0,
+                        kDefaultWaitTimeoutNs, block_mask);
     } catch (...) {
         return VDIT_ERR_CUDA;
     }

@@ -9,7 +9,7 @@ figure in "Realtime video generation: FLOPS calculation and optimizations"
 """
 from __future__ import annotations
 
-from .workloads import MASK_BLOCK_CAUSAL, Attn
+from .workloads import MASK_BLOCK_CAUSAL, MASK_BLOCK_SPARSE, SPARSE_BLOCK, Attn
 
 
 def allowed_pairs(Sq: int, Skv: int, mask_kind: int, chunk_tokens: int = 0) -> int:
@@ -24,8 +24,20 @@ def allowed_pairs(Sq: int, Skv: int, mask_kind: int, chunk_tokens: int = 0) -> i
     return Sq * Skv
 
 
-def attn_flops(call: Attn) -> float:
+def sparse_allowed_pairs(block_mask, Sq: int, Skv: int) -> int:
+    """Allowed (query, key) pairs of a [B, H, nqb, nkb] block mask, summed over B and H."""
+    import numpy as np
+    m = np.asarray(block_mask) != 0
+    nqb, nkb = m.shape[-2], m.shape[-1]
+    rows = np.minimum(SPARSE_BLOCK, Sq - SPARSE_BLOCK * np.arange(nqb))  # tokens per query block
+    cols = np.minimum(SPARSE_BLOCK, Skv - SPARSE_BLOCK * np.arange(nkb))
+    return int(np.einsum("bhqk,q,k->", m.astype(np.int64), rows, cols))
+
+
+def attn_flops(call: Attn, block_mask=None) -> float:
     """Algorithmic FLOPs of one call: 2*D for QK^T plus 2*D for PV per pair."""
+    if call.mask_kind == MASK_BLOCK_SPARSE:
+        return 4.0 * call.D * sparse_allowed_pairs(block_mask, call.Sq, call.Skv)
     return 4.0 * call.B * call.H * call.D * allowed_pairs(
         call.Sq, call.Skv, call.mask_kind, call.chunk_tokens)
 

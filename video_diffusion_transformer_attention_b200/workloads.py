@@ -36,6 +36,8 @@ import torch
 MASK_FULL = 0
 MASK_BLOCK_CAUSAL = 1
 MASK_CROSS = 2
+MASK_BLOCK_SPARSE = 3
+SPARSE_BLOCK = 128
 
 RMS_EPS = 1e-6
 OUTLIER_CHANNELS = 3  # round(0.02 * 128)
@@ -87,7 +89,15 @@ WORKLOADS = {
     "block_causal_7x4680": Workload(
         "block_causal_7x4680", 4, "rms_qk",
         (Attn("self", 1, 12, 32760, 32760, 128, MASK_BLOCK_CAUSAL, 4680),)),
+    # block-sparse self-attention on the 720p Wan2.1-14B shape: each query
+    # block keeps its own key block plus a seeded 25% of the others (the
+    # page's "x4" for block-sparse attention read as keeping a quarter)
+    "wan21_14b_720p_sparse25": Workload(
+        "wan21_14b_720p_sparse25", 5, "rms_qk",
+        (Attn("self", 1, 40, 75600, 75600, 128, MASK_BLOCK_SPARSE),)),
 }
+
+SPARSE_DENSITY = 0.25
 
 
 def _rms_normalise(x: torch.Tensor) -> torch.Tensor:
@@ -143,12 +153,32 @@ def workload_inputs(name: str):
     q, k, v = draw_qkv(self_call.B, self_call.H, self_call.Sq, self_call.Skv,
                        self_call.D, 1000 + w.index, w.recipe)
     out = {"q": q, "k": k, "v": v}
+    if self_call.mask_kind == MASK_BLOCK_SPARSE:
+        out["block_mask"] = draw_block_mask(self_call.B, self_call.H, self_call.Sq, self_call.Skv,
+                                            SPARSE_DENSITY, 3000 + w.index)
     if w.text_tokens:
         kt, vt = draw_text_kv(self_call.B, self_call.H, w.text_tokens,
                               self_call.D, 2000 + w.index)
         out["k_text"] = kt
         out["v_text"] = vt
     return out
+
+
+def draw_block_mask(B: int, H: int, Sq: int, Skv: int, density: float, seed: int,
+                    keep_diagonal: bool = True) -> torch.Tensor:
+    """Seeded block mask [B, H, ceil(Sq/128), ceil(Skv/128)] uint8 (CPU).
+
+    Each block is kept with probability `density`; with keep_diagonal the
+    block pair (i, i) is always kept (a query block sees its own tokens).
+    """
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(int(seed))
+    nqb, nkb = -(-Sq // SPARSE_BLOCK), -(-Skv // SPARSE_BLOCK)
+    m = (torch.rand((B, H, nqb, nkb), generator=gen) < density)
+    if keep_diagonal:
+        d = torch.arange(min(nqb, nkb))
+        m[:, :, d, d] = True
+    return m.to(torch.uint8)
 
 
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
