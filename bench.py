@@ -392,6 +392,40 @@ def run_vdit(args):
     return 0
 
 
+def run_merge(args):
+    """Time vdit_attn_merge at the self-attention shape of the workload (HBM-bound)."""
+    from video_diffusion_transformer_attention_b200 import binding as vb
+    dev = torch.device("cuda", 0)
+    call = wl.WORKLOADS[args.workload].calls[0]
+    B, H, S, D = call.B, call.H, call.Sq, call.D
+    o_acc = torch.randn(B, S, H, D, device=dev).to(torch.bfloat16)
+    o_part = torch.randn(B, S, H, D, device=dev).to(torch.bfloat16)
+    lse_acc = torch.randn(B, H, S, device=dev)
+    lse_part = torch.randn(B, H, S, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    sp = int(stream.cuda_stream)
+    for _ in range(args.warmup):
+        vb.vdit_attn_merge(o_acc, lse_acc, o_part, lse_part, B, H, S, D, sp)
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        vb.vdit_attn_merge(o_acc, lse_acc, o_part, lse_part, B, H, S, D, sp)
+    e1.record(stream)
+    stream.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    rows = B * H * S
+    nbytes = rows * (3 * D * 2 + 3 * 4)  # read two O rows and two LSE, write one of each
+    peaks, src = load_peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    print(json.dumps({"kernel": "attn_merge_kernel", "workload": f"{args.workload} B={B} H={H} S={S} D={D}",
+                      "ms": ms, "bytes": nbytes,
+                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                   "frac": gbs / peaks["hbm_gbs"], "peak_kind": f"{src} copy bandwidth"}}),
+          flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -402,11 +436,15 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--reference-seconds", type=float, default=40.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=("attention", "merge"), default="attention",
+                    help="merge: time only the LSE merge kernel (HBM roofline)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "vdit":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         return run_reference(args)
+    if args.kernel == "merge":
+        return run_merge(args)
     return run_vdit(args)
 
 

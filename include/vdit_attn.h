@@ -143,6 +143,27 @@ vdit_status vdit_attn_fwd_ws(const void* q, const void* k, const void* v,
                              size_t workspace_bytes, void* stream);
 
 /*
+ * vdit_attn_merge -- fold a partial attention result into a running one.
+ * For each (b, h, i), with (o_acc, lse_acc) attention over one key set and
+ * (o_part, lse_part) over a disjoint key set, writes attention over their
+ * union into (o_acc, lse_acc):
+ *   LSE = ln(e^lse_acc + e^lse_part),
+ *   O   = e^(lse_acc - LSE) o_acc + e^(lse_part - LSE) o_part.
+ * This is the combine step of ring context parallelism over K/V blocks (the
+ * Wave Forcing digest (airadar.tv) compares Wave Parallelism with Ulysses and
+ * Ring context parallelism); it is why vdit_attn_fwd returns LSE.
+ *   o_acc, o_part     : device bf16 [B][S][H][D] (BSHD), D == 128
+ *   lse_acc, lse_part : device fp32 [B][H][S], natural log
+ * A row with lse = -inf contributes nothing; two -inf rows give O = 0,
+ * LSE = -inf.  fp32 arithmetic, O rounded to bf16.  Buffers must not overlap
+ * (except that o_acc and lse_acc are read and written in place); pointers
+ * 16-byte aligned.  Asynchronous on `stream`.
+ */
+vdit_status vdit_attn_merge(void* o_acc, float* lse_acc, const void* o_part,
+                            const float* lse_part, int B, int H, int S, int D,
+                            void* stream);
+
+/*
  * vdit_get_device_status -- synchronises `stream`, then reads and clears the
  * current device's error word that the kernels set when a bounded wait on
  * one of their pipeline barriers runs out.  Returns VDIT_OK,

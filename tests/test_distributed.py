@@ -4,6 +4,7 @@ The forward shards with no exchange: each rank runs its own problem and the
 benchmark only reduces its timing with a max over ranks.  These tests run that
 reduction and the rank handling of the reference arm without a GPU.
 """
+import math
 import os
 import socket
 import subprocess
@@ -64,3 +65,90 @@ def test_reference_arm_exits_quietly_on_nonzero_rank():
                         "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0
     assert r.stdout.strip() == ""
+
+
+# ---------------------------------------------------------------- context parallel schedules
+
+def _fake_attn(q, k, v):
+    """Stand-in for the CUDA attention with Q = 0 semantics: O = mean of the V
+    rows, LSE = ln(#keys).  Exercises only the schedule, not the arithmetic."""
+    B, Sq, H, D = q.shape
+    n = k.shape[1]
+    o = v.double().mean(dim=1, keepdim=True).expand(B, Sq, H, D).contiguous()
+    lse = torch.full((B, H, Sq), math.log(n), dtype=torch.float64)
+    return o, lse
+
+
+def _fake_merge(o_acc, lse_acc, o_part, lse_part):
+    lse = torch.logaddexp(lse_acc, lse_part)
+    wa = torch.exp(lse_acc - lse).permute(0, 2, 1)[..., None]
+    wp = torch.exp(lse_part - lse).permute(0, 2, 1)[..., None]
+    o_acc.copy_(wa * o_acc + wp * o_part)
+    lse_acc.copy_(lse)
+
+
+def _ring_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    from video_diffusion_transformer_attention_b200 import parallel
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        gen = torch.Generator().manual_seed(7)
+        B, S_local, H, D = 1, 5, 3, 8
+        v_all = torch.randn(world, B, S_local, H, D, generator=gen, dtype=torch.float64)
+        q = torch.zeros(B, 4, H, D, dtype=torch.float64)
+        k = torch.zeros(B, S_local, H, D, dtype=torch.float64)
+        v = v_all[rank].contiguous()
+        o, lse = parallel.ring_attention(q, k, v, attn=_fake_attn, merge=_fake_merge)
+        expect = v_all.permute(1, 0, 2, 3, 4).reshape(B, world * S_local, H, D).mean(dim=1)
+        out[rank] = (float((o - expect[:, None]).abs().max()), float((lse - math.log(world * S_local)).abs().max()))
+    finally:
+        dist.destroy_process_group()
+
+
+def _ulysses_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    from video_diffusion_transformer_attention_b200 import parallel
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        gen = torch.Generator().manual_seed(3)
+        B, S, H, D = 2, 6, 4, 8
+        full = torch.randn(B, S, H, D, generator=gen)
+        s = S // world
+        shard = full[:, rank * s:(rank + 1) * s].contiguous()
+        heads = parallel.seq_to_head_shards(shard)
+        hs = H // world
+        ok_heads = torch.equal(heads, full[:, :, rank * hs:(rank + 1) * hs])
+        back = parallel.head_to_seq_shards(heads)
+        ok_back = torch.equal(back, shard)
+        # full pass with an identity "attention": output = the query shard again
+        o, _ = parallel.ulysses_attention(shard, shard, shard, attn=lambda q, k, v: (q, None))
+        out[rank] = (ok_heads, ok_back, torch.equal(o, shard))
+    finally:
+        dist.destroy_process_group()
+
+
+def _spawn(target, world=2):
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = free_port()
+    procs = [ctx.Process(target=target, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    return dict(out)
+
+
+def test_ring_schedule_visits_every_kv_shard_once():
+    out = _spawn(_ring_worker)
+    for rank, (err_o, err_lse) in out.items():
+        assert err_o < 1e-12 and err_lse < 1e-12, (rank, err_o, err_lse)
+
+
+def test_ulysses_all_to_all_layouts():
+    out = _spawn(_ulysses_worker)
+    assert all(all(v) for v in out.values()), out

@@ -38,6 +38,7 @@ EXPORTS = (
     "vdit_attn_fwd",
     "vdit_attn_fwd_ws",
     "vdit_attn_fwd_block_sparse",
+    "vdit_attn_merge",
     "vdit_get_device_status",
     "vdit_status_string",
     "vdit_abi_version",
@@ -77,6 +78,8 @@ def lib() -> ctypes.CDLL:
             h.vdit_attn_fwd_block_sparse.restype = c_int
             h.vdit_attn_fwd_block_sparse.argtypes = [vp, vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int,
                                                      c_float, vp]
+            h.vdit_attn_merge.restype = c_int
+            h.vdit_attn_merge.argtypes = [vp, vp, vp, vp, c_int, c_int, c_int, c_int, vp]
             h.vdit_testing_attn_fwd.restype = c_int
             h.vdit_testing_attn_fwd.argtypes = fwd_args + [c_int, ctypes.c_ulonglong, vp]
             h.vdit_get_device_status.restype = c_int
@@ -153,6 +156,15 @@ def vdit_attn_fwd_block_sparse(q, k, v, o, lse, block_mask, B, H, Sq, Skv, D, sc
                                           B, H, Sq, Skv, D, float(scale), _stream(stream))
     if check and st != VDIT_OK:
         raise VditError(st, "vdit_attn_fwd_block_sparse")
+    return st
+
+
+def vdit_attn_merge(o_acc, lse_acc, o_part, lse_part, B, H, S, D, stream=None, check=True) -> int:
+    """Fold (o_part, lse_part) into (o_acc, lse_acc) in place (see include/vdit_attn.h)."""
+    st = lib().vdit_attn_merge(_addr(o_acc), _addr(lse_acc), _addr(o_part), _addr(lse_part), B, H, S, D,
+                               _stream(stream))
+    if check and st != VDIT_OK:
+        raise VditError(st, "vdit_attn_merge")
     return st
 
 

@@ -15,6 +15,7 @@
 #include "vdit_attn.h"
 #include "vdit_attn_testing.h"
 #include "attn_fwd_sm100.cuh"
+#include "attn_merge.cuh"
 
 namespace {
 
@@ -269,6 +270,37 @@ vdit_status vdit_testing_attn_fwd(const void* q, const void* k, const void* v, v
         const int flags = fault == VDIT_TESTING_WITHHOLD_KV ? vdit::kDebugWithholdKV : 0;
         return fwd_impl(q, k, v, o, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, nullptr, 0, stream, flags,
                         wait_timeout_ns);
+    } catch (...) {
+        return VDIT_ERR_CUDA;
+    }
+}
+
+vdit_status vdit_attn_merge(void* o_acc, float* lse_acc, const void* o_part, const float* lse_part, int B, int H,
+                            int S, int D, void* stream) {
+    try {
+        if (B < 0 || H < 0 || S < 0 || D < 1) return VDIT_ERR_INVALID_ARG;
+        if (D != vdit::kHeadDim) return VDIT_ERR_UNSUPPORTED;
+        if (B == 0 || H == 0 || S == 0) return VDIT_OK;
+        if (o_acc == nullptr || lse_acc == nullptr || o_part == nullptr || lse_part == nullptr)
+            return VDIT_ERR_INVALID_ARG;
+        if (!aligned16(o_acc) || !aligned16(o_part) || !aligned16(lse_acc) || !aligned16(lse_part))
+            return VDIT_ERR_MISALIGNED;
+        const long long rows = (long long)B * S * H;
+        const long long blocks = (rows + vdit::kMergeWarpsPerBlock - 1) / vdit::kMergeWarpsPerBlock;
+        if (blocks > 0x7fffffffLL) return VDIT_ERR_INVALID_ARG;
+        const size_t o_bytes = size_t(rows) * size_t(D) * 2, l_bytes = size_t(rows) * 4;
+        if (overlaps(o_acc, o_bytes, o_part, o_bytes) || overlaps(lse_acc, l_bytes, lse_part, l_bytes) ||
+            overlaps(o_acc, o_bytes, lse_acc, l_bytes) || overlaps(o_acc, o_bytes, lse_part, l_bytes) ||
+            overlaps(lse_acc, l_bytes, o_part, o_bytes))
+            return VDIT_ERR_INVALID_ARG;
+        int sm_count = 0;
+        const vdit_status st = ensure_device(&sm_count);
+        if (st != VDIT_OK) return st;
+        vdit::attn_merge_kernel<<<unsigned(blocks), vdit::kMergeWarpsPerBlock * 32, 0,
+                                  static_cast<cudaStream_t>(stream)>>>(
+            static_cast<__nv_bfloat16*>(o_acc), lse_acc, static_cast<const __nv_bfloat16*>(o_part), lse_part, B, H,
+            S);
+        return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
     } catch (...) {
         return VDIT_ERR_CUDA;
     }
