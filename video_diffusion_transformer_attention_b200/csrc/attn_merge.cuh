@@ -10,9 +10,12 @@
 // attends to one K/V block and folds the partial result into the running one.
 // An empty partial (LSE = -inf) leaves the other unchanged.
 //
-// HBM-bound: one warp per (b, i, h) row, each lane 4 of the 128 head dims
-// (8-byte loads and stores, coalesced 256 B per warp); per row it reads two
-// O rows and two LSE values and writes one of each.
+// HBM-bound.  A warp takes 32 consecutive query rows i of one (b, h): each
+// lane reads the two LSE values of one row (coalesced) and computes that
+// row's merge weights once, then the warp walks the 32 rows, every lane
+// handling 4 of the 128 head dims (8-byte accesses, 256 B per row), with the
+// weights broadcast by shuffle.  Per row it reads two O rows and two LSE
+// values and writes one of each.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -21,48 +24,72 @@
 namespace vdit {
 
 constexpr int kMergeWarpsPerBlock = 8;
+constexpr int kMergeRowsPerWarp = 32;
 
 __global__ void __launch_bounds__(kMergeWarpsPerBlock * 32)
     attn_merge_kernel(__nv_bfloat16* __restrict__ o_acc, float* __restrict__ lse_acc,
                       const __nv_bfloat16* __restrict__ o_part, const float* __restrict__ lse_part, int B, int H,
                       int S) {
-    const long long rows = static_cast<long long>(B) * S * H;
-    const long long r = static_cast<long long>(blockIdx.x) * kMergeWarpsPerBlock + (threadIdx.x >> 5);
-    if (r >= rows) return;
     const int lane = threadIdx.x & 31;
-    // O row r = (b * S + i) * H + h; LSE index (b * H + h) * S + i
-    const long long bs = r / H;
-    const int h = static_cast<int>(r - bs * H);
-    const long long b = bs / S;
-    const int i = static_cast<int>(bs - b * S);
-    const long long li = (b * H + h) * S + i;
-    const float la = lse_acc[li];
-    const float lp = lse_part[li];
-    const float mx = fmaxf(la, lp);
-    float wa = 0.0f, wp = 0.0f, lse = -INFINITY;
-    if (mx != -INFINITY) {
-        const float ea = expf(la - mx);
-        const float ep = expf(lp - mx);
-        const float sum = ea + ep;
-        wa = ea / sum;
-        wp = ep / sum;
-        lse = mx + logf(sum);
+    const long long chunks = (S + kMergeRowsPerWarp - 1) / kMergeRowsPerWarp;
+    const long long wid = static_cast<long long>(blockIdx.x) * kMergeWarpsPerBlock + (threadIdx.x >> 5);
+    if (wid >= static_cast<long long>(B) * H * chunks) return;
+    const long long bh = wid / chunks;  // b * H + h
+    const int i0 = static_cast<int>(wid - bh * chunks) * kMergeRowsPerWarp;
+    const int b = static_cast<int>(bh / H);
+    const int h = static_cast<int>(bh - static_cast<long long>(b) * H);
+    const int n = min(kMergeRowsPerWarp, S - i0);
+
+    // lane l: weights of row i0 + l
+    float wa = 0.0f, wp = 0.0f;
+    if (lane < n) {
+        const long long li = bh * S + i0 + lane;
+        const float la = lse_acc[li];
+        const float lp = lse_part[li];
+        const float mx = fmaxf(la, lp);
+        float lse = -INFINITY;
+        if (mx != -INFINITY) {
+            const float ea = expf(la - mx);
+            const float ep = expf(lp - mx);
+            const float inv = 1.0f / (ea + ep);
+            wa = ea * inv;
+            wp = ep * inv;
+            lse = mx + logf(ea + ep);
+        }
+        lse_acc[li] = lse;
     }
-    const size_t off = static_cast<size_t>(r) * 128 + lane * 4;
-    const uint2 a = *reinterpret_cast<const uint2*>(o_acc + off);
-    const uint2 p = *reinterpret_cast<const uint2*>(o_part + off);
-    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
-    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&p);
-    uint2 out;
-    __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&out);
+    // O row (b, i, h) at ((b * S + i) * H + h) * 128
+    const size_t row0 = (static_cast<size_t>(b) * S + i0) * H + h;
+    const size_t stride = static_cast<size_t>(H) * 128;
+    for (int r0 = 0; r0 < n; r0 += 4) {
+        uint2 a[4], p[4];
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        const float2 fa = __bfloat1622float2(a2[k]);
-        const float2 fp = __bfloat1622float2(p2[k]);
-        o2[k] = __floats2bfloat162_rn(wa * fa.x + wp * fp.x, wa * fa.y + wp * fp.y);
+        for (int u = 0; u < 4; ++u) {
+            if (r0 + u < n) {
+                const size_t off = (row0 * 128) + (r0 + u) * stride + lane * 4;
+                a[u] = *reinterpret_cast<const uint2*>(o_acc + off);
+                p[u] = __ldg(reinterpret_cast<const uint2*>(o_part + off));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float ra = __shfl_sync(0xffffffffu, wa, (r0 + u) & 31);
+            const float rp = __shfl_sync(0xffffffffu, wp, (r0 + u) & 31);
+            if (r0 + u < n) {
+                const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a[u]);
+                const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&p[u]);
+                uint2 out;
+                __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&out);
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const float2 fa = __bfloat1622float2(a2[k]);
+                    const float2 fp = __bfloat1622float2(p2[k]);
+                    o2[k] = __floats2bfloat162_rn(ra * fa.x + rp * fp.x, ra * fa.y + rp * fp.y);
+                }
+                *reinterpret_cast<uint2*>(o_acc + (row0 * 128) + (r0 + u) * stride + lane * 4) = out;
+            }
+        }
     }
-    *reinterpret_cast<uint2*>(o_acc + off) = out;
-    if (lane == 0) lse_acc[li] = lse;
 }
 
 }  // namespace vdit

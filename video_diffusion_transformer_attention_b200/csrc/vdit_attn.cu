@@ -286,7 +286,8 @@ vdit_status vdit_attn_merge(void* o_acc, float* lse_acc, const void* o_part, con
         if (!aligned16(o_acc) || !aligned16(o_part) || !aligned16(lse_acc) || !aligned16(lse_part))
             return VDIT_ERR_MISALIGNED;
         const long long rows = (long long)B * S * H;
-        const long long blocks = (rows + vdit::kMergeWarpsPerBlock - 1) / vdit::kMergeWarpsPerBlock;
+        const long long warps = (long long)B * H * ((S + vdit::kMergeRowsPerWarp - 1) / vdit::kMergeRowsPerWarp);
+        const long long blocks = (warps + vdit::kMergeWarpsPerBlock - 1) / vdit::kMergeWarpsPerBlock;
         if (blocks > 0x7fffffffLL) return VDIT_ERR_INVALID_ARG;
         const size_t o_bytes = size_t(rows) * size_t(D) * 2, l_bytes = size_t(rows) * 4;
         if (overlaps(o_acc, o_bytes, o_part, o_bytes) || overlaps(lse_acc, l_bytes, lse_part, l_bytes) ||
