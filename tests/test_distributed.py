@@ -152,3 +152,31 @@ def test_ring_schedule_visits_every_kv_shard_once():
 def test_ulysses_all_to_all_layouts():
     out = _spawn(_ulysses_worker)
     assert all(all(v) for v in out.values()), out
+
+
+def _dead_peer_worker(rank, world, port, out):
+    import datetime
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    from video_diffusion_transformer_attention_b200 import parallel
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        out[rank] = "left"
+        os._exit(0)  # leaves between steps, without tearing down the group
+    q = torch.zeros(1, 4, 2, 8, dtype=torch.float64)
+    k = torch.zeros(1, 3, 2, 8, dtype=torch.float64)
+    v = torch.ones(1, 3, 2, 8, dtype=torch.float64)
+    import time
+    t0 = time.time()
+    try:
+        parallel.ring_attention(q, k, v, attn=_fake_attn, merge=_fake_merge)
+        out[rank] = "no error"
+    except Exception as e:  # the exchange with the departed rank must fail, not hang
+        out[rank] = f"error after {time.time() - t0:.1f}s: {type(e).__name__}"
+
+
+def test_a_departed_rank_makes_the_ring_fail_instead_of_hang():
+    out = _spawn(_dead_peer_worker)
+    assert out[1] == "left"
+    assert out[0].startswith("error after"), out[0]
+    assert float(out[0].split()[2][:-2]) < 60

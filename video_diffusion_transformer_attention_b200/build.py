@@ -52,7 +52,7 @@ def check_launch_registers(ptxas_log: str) -> int:
     """The forward kernel re-splits its registers with setmaxnreg, which is only
     safe if ptxas allocated exactly kLaunchRegs a thread at launch; a smaller
     allocation would leave setmaxnreg.inc waiting forever.  Returns the count."""
-    found = re.findall(r"Compiling entry function '(\w*attn_fwd_sm100_kernel\w*)'.*?Used (\d+) registers",
+    found = re.findall(r"Compiling entry function '(\w*attn_fwd_\w*kernel\w*)'.*?Used (\d+) registers",
                        ptxas_log, flags=re.S)
     if not found:
         raise RuntimeError("could not find the forward kernel's register count in the ptxas output")
