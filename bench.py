@@ -250,7 +250,9 @@ def run_vdit(args):
 
     vb.lib()
     w, desc = workload_config(args.workload)
-    inp_cpu = wl.workload_inputs(args.workload)
+    # --qknorm: Q and K are drawn raw; the self-attention call normalises them
+    # (per-head RMS norm into a workspace) and then attends
+    inp_cpu = wl.workload_inputs(args.workload, raw_qk=args.qknorm)
     inp = {k: v.to(dev) for k, v in inp_cpu.items()}
     outs = []
     for call in w.calls:
@@ -261,9 +263,20 @@ def run_vdit(args):
     mask_cpu = inp_cpu.get("block_mask")
     flops_per_call = [fl.attn_flops(c, mask_cpu) for c in w.calls]
     step_flops = sum(flops_per_call)
+    qk_ws = None
+    if args.qknorm:
+        c0 = w.calls[0]
+        st, need = vb.vdit_attn_qknorm_plan(c0.B, c0.H, c0.Sq, c0.Skv, c0.D, c0.mask_kind, c0.chunk_tokens)
+        if st != vb.VDIT_OK:
+            raise SystemExit(f"vdit_attn_qknorm_plan: {vb.vdit_status_string(st)}")
+        qk_ws = torch.empty(need, dtype=torch.uint8, device=dev)
 
     def launch(i, call, q, k, v, o, lse):
-        if call.mask_kind == wl.MASK_BLOCK_SPARSE:
+        if args.qknorm and call.name == "self":
+            vb.vdit_attn_fwd_qknorm(q, k, v, o, lse, None, None, wl.RMS_EPS, call.B, call.H, call.Sq, call.Skv,
+                                    call.D, call.scale, call.mask_kind, call.chunk_tokens, qk_ws, qk_ws.numel(),
+                                    sptr)
+        elif call.mask_kind == wl.MASK_BLOCK_SPARSE:
             vb.vdit_attn_fwd_block_sparse(q, k, v, o, lse, inp["block_mask"], call.B, call.H, call.Sq, call.Skv,
                                           call.D, call.scale, sptr)
         else:
@@ -363,12 +376,15 @@ def run_vdit(args):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"{args.workload} ({desc})", "l2": "inputs larger than L2 (3.1 GB per step)",
+            "config": {"workload": f"{args.workload} ({desc})" + (" [raw Q/K: per-head RMS norm + attention]"
+                                                                  if args.qknorm else ""),
+                       "l2": "inputs larger than L2 (3.1 GB per step)",
                        "parallelism": f"independent replicas x{world} (no collective)"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_sustained, "unit": "TFLOP/s",
                          "frac": achieved / peak_sustained,
                          "traffic": recorded_traffic() if args.workload == WORKLOAD else None,
-                         "kernel": "attn_fwd_sm100_kernel (self-attention launch)",
+                         "kernel": "attn_fwd_sm100_kernel (self-attention launch)" if not args.qknorm else
+                                   "qk_rms_norm_kernel + attn_fwd_sm100_kernel (self-attention call)",
                          "peak_kind": f"{peak_src} sustained bf16 (cuBLAS, power-capped)",
                          "frac_of_burst": achieved / peak_burst,
                          "frac_of_datasheet": achieved / DATASHEET_BF16_TFLOPS},
@@ -436,6 +452,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--reference-seconds", type=float, default=40.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--qknorm", action="store_true",
+                    help="raw Q/K with the per-head RMS norm fused into the self-attention call")
     ap.add_argument("--kernel", choices=("attention", "merge"), default="attention",
                     help="merge: time only the LSE merge kernel (HBM roofline)")
     args = ap.parse_args()

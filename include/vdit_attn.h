@@ -132,6 +132,61 @@ vdit_status vdit_attn_fwd_block_sparse(const void* q, const void* k,
                                        void* stream);
 
 /*
+ * vdit_qk_rms_norm -- per-head RMS norm of the query and key tensors, in one
+ * launch:
+ *     y[b,s,h,:] = x * rsqrt(mean_d(x^2) + eps) * w[h][:]   (fp32, rounded to bf16)
+ * for x the rows of q (weight q_norm_weight) and of k (k_norm_weight).  This
+ * is the query/key normalisation of the Wan2.x blocks that the gonka
+ * DiT-support discussion (#1155) proposes to serve; its "Pricing policy"
+ * section counts normalisation among the parts of a forward pass that grow
+ * linearly with the number of latent patches.
+ *   q, k          : device bf16 [B][Sq][H][D] and [B][Skv][H][D]; either may
+ *                   be absent (NULL) when its token count is 0.
+ *   q_out, k_out  : device bf16, same shapes; each is either exactly its
+ *                   input (in place) or overlaps no other buffer.
+ *   q_norm_weight, k_norm_weight : device fp32 [H][D], or NULL for all ones.
+ *   eps           : finite and > 0.
+ * D must be 128; every pointer 16-byte aligned (VDIT_ERR_MISALIGNED).
+ * Asynchronous on `stream`; HBM-bound (256 bytes read and written per row).
+ */
+vdit_status vdit_qk_rms_norm(const void* q, const void* k, void* q_out,
+                             void* k_out, const float* q_norm_weight,
+                             const float* k_norm_weight, float eps, int B,
+                             int H, int Sq, int Skv, int D, void* stream);
+
+/*
+ * vdit_attn_qknorm_plan -- host-only: the workspace size, in bytes, that
+ * vdit_attn_fwd_qknorm needs for this shape (the normalised Q and K).
+ * Same shape rules as vdit_attn_plan; VDIT_MASK_BLOCK_SPARSE is not
+ * accepted.
+ */
+vdit_status vdit_attn_qknorm_plan(int B, int H, int Sq, int Skv, int D,
+                                  int mask_kind, int chunk_tokens,
+                                  size_t* workspace_bytes);
+
+/*
+ * vdit_attn_fwd_qknorm -- vdit_attn_fwd on raw Q and K: first
+ * vdit_qk_rms_norm of q and k into `workspace`, then the attention on the
+ * normalised tensors, queued as a programmatic dependent launch so that its
+ * CTAs start while the norm drains (its loads of Q and K wait for the norm
+ * to complete).  q and k are not modified.
+ *   q_norm_weight, k_norm_weight, eps : as vdit_qk_rms_norm.
+ *   workspace     : caller-owned device memory of at least the size
+ *                   vdit_attn_qknorm_plan reports, 256-byte aligned, not
+ *                   overlapping any other argument (VDIT_ERR_WORKSPACE when
+ *                   NULL or too small).
+ * Other arguments as vdit_attn_fwd; VDIT_MASK_BLOCK_SPARSE is not accepted
+ * (normalise with vdit_qk_rms_norm, then call vdit_attn_fwd_block_sparse).
+ */
+vdit_status vdit_attn_fwd_qknorm(const void* q, const void* k, const void* v,
+                                 void* o, float* lse, const float* q_norm_weight,
+                                 const float* k_norm_weight, float eps, int B,
+                                 int H, int Sq, int Skv, int D, float scale,
+                                 int mask_kind, int chunk_tokens,
+                                 void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/*
  * vdit_attn_fwd_ws -- vdit_attn_fwd with a caller-owned device workspace of
  * `workspace_bytes` bytes (at least what vdit_attn_plan reports; NULL is
  * accepted when that is 0).

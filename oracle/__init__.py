@@ -12,5 +12,7 @@ from .oracle import (  # noqa: F401
     attention,
     build,
     max_threads,
+    rms_norm,
+    round_to_bf16_bits,
     SPARSE_BLOCK,
 )

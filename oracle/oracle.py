@@ -122,3 +122,41 @@ def attention(q_bits, k_bits, v_bits, scale: float, mask_kind: int = MASK_FULL,
         o = o.reshape(B, H, Sq, D).transpose(0, 2, 1, 3).copy()
         lse = lse.reshape(B, H, Sq)
     return o, lse
+
+
+def round_to_bf16_bits(x) -> np.ndarray:
+    """Round float64 values to the nearest bf16 (ties to even); returns the bit patterns.
+
+    bf16 keeps 8 significant bits: with x = m * 2^e, 0.5 <= |m| < 1, the
+    rounded value is rint(m * 2^8) * 2^(e - 8), where rint rounds half to even.
+    Finite, normal-range inputs only (the RMS-normalised tensors this serves).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)
+    r = np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)   # exactly representable in binary32
+    return (r.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def rms_norm(x_bits, weight=None, eps: float = 1e-6) -> np.ndarray:
+    """Per-(token, head) RMS norm of a bf16 [B, S, H, D] tensor, in float64.
+
+    y[b, s, h, :] = x / sqrt(mean_d(x^2) + eps) * weight[h, :]  (weight None = 1).
+
+    The pages name normalisation only as one of the parts of a DiT forward
+    pass whose cost grows linearly with the latent patch count (gonka
+    discussion #1155 on DiT support, "Pricing policy").  Read here as the
+    per-head query/key RMS norm of the Wan2.x blocks that page proposes to
+    serve: one learned weight per (head, channel), applied right before
+    attention.  The attention then takes the result rounded to bf16
+    (round_to_bf16_bits), the operand type of its bf16 products.
+    """
+    a = _as_bits(x_bits)
+    x = (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    y = x / np.sqrt(ms + eps)
+    if weight is not None:
+        w = np.asarray(weight, dtype=np.float64)
+        if w.shape != a.shape[2:]:
+            raise ValueError("weight is [H, D]")
+        y = y * w
+    return y

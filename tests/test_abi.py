@@ -114,6 +114,41 @@ def test_block_sparse_needs_its_entry_point_and_a_mask():
                                          check=False) == vb.VDIT_ERR_UNSUPPORTED
 
 
+def test_qknorm_entry_point_argument_checks():
+    args = (A, A * 3, A * 5, A * 7, A * 9)
+    ok_shape = (1, 2, 64, 64, 128, 0.1)
+    ws = A * 64
+    st, need = vb.vdit_attn_qknorm_plan(1, 2, 64, 64, 128, 0, 0)
+    assert st == vb.VDIT_OK and need == 64 * 2 * 128 * 2 * 2   # normalised Q and K, Q rounded up to 256 B
+    assert vb.vdit_attn_qknorm_plan(1, 2, 64, 64, 128, vb.VDIT_MASK_BLOCK_SPARSE, 0)[0] == vb.VDIT_ERR_INVALID_ARG
+    assert vb.vdit_attn_qknorm_plan(1, 2, 64, 64, 64, 0, 0)[0] == vb.VDIT_ERR_UNSUPPORTED
+
+    def call(*extra, eps=1e-6, qw=None, mask=0, workspace=ws, nbytes=need):
+        return vb.vdit_attn_fwd_qknorm(*args, qw, None, eps, *ok_shape, mask, 0, workspace, nbytes, stream=0,
+                                       check=False)
+    assert call(eps=0.0) == vb.VDIT_ERR_INVALID_ARG                     # eps must be > 0
+    assert call(eps=float("nan")) == vb.VDIT_ERR_INVALID_ARG
+    assert call(mask=vb.VDIT_MASK_BLOCK_SPARSE) == vb.VDIT_ERR_INVALID_ARG
+    assert call(qw=A * 11 + 4) == vb.VDIT_ERR_MISALIGNED
+    assert call(workspace=None) == vb.VDIT_ERR_WORKSPACE
+    assert call(nbytes=need - 1) == vb.VDIT_ERR_WORKSPACE
+    assert call(workspace=ws + 16) == vb.VDIT_ERR_MISALIGNED            # 256-byte alignment
+    assert call(workspace=A) == vb.VDIT_ERR_INVALID_ARG                 # overlaps q
+
+
+def test_qk_rms_norm_argument_checks():
+    def call(q=A, k=A * 3, qo=A * 5, ko=A * 7, eps=1e-6, D=128, Sq=64, Skv=64, qw=None):
+        return vb.vdit_qk_rms_norm(q, k, qo, ko, qw, None, eps, 1, 2, Sq, Skv, D, stream=0, check=False)
+    assert call(eps=-1.0) == vb.VDIT_ERR_INVALID_ARG
+    assert call(D=64) == vb.VDIT_ERR_UNSUPPORTED
+    assert call(qo=A * 5 + 8) == vb.VDIT_ERR_MISALIGNED
+    assert call(qw=A * 9 + 4) == vb.VDIT_ERR_MISALIGNED
+    assert call(qo=A + 256) == vb.VDIT_ERR_INVALID_ARG                  # partial overlap with its input
+    assert call(ko=A * 5) == vb.VDIT_ERR_INVALID_ARG                    # the two outputs overlap
+    assert call(k=None, Skv=64) == vb.VDIT_ERR_INVALID_ARG
+    assert call(Sq=0, Skv=0) == vb.VDIT_OK                              # nothing to do, nothing launched
+
+
 def test_empty_call_is_a_no_op():
     for B, H, Sq in [(0, 2, 64), (1, 0, 64), (1, 2, 0)]:
         assert vb.vdit_attn_fwd(None, None, None, None, None, B, H, Sq, 64, 128, 0.1, 0, 0,

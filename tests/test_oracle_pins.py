@@ -302,3 +302,55 @@ def test_block_sparse_rejects_a_wrong_mask_shape():
     qb = np.zeros((1, 200, 1, 8), np.uint16)
     with pytest.raises(ValueError):
         attention(qb, qb, qb, 0.5, MASK_BLOCK_SPARSE, block_mask=np.ones((1, 1, 1, 1)))
+
+
+# ---------------------------------------------------------------------------
+# Per-head Q/K RMS norm (the fused prologue's reference) and bf16 rounding.
+# ---------------------------------------------------------------------------
+from oracle import rms_norm, round_to_bf16_bits  # noqa: E402
+
+
+def test_bf16_rounding_matches_torch_cast_and_ties_go_to_even():
+    g = torch.Generator().manual_seed(31)
+    x = torch.randn(4096, generator=g, dtype=torch.float32) * 7.0
+    want = x.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(round_to_bf16_bits(x.double().numpy()), want)
+    ulp = 2.0 ** -7                               # bf16 spacing in [1, 2)
+    ties = np.array([1 + ulp / 2, 1 + 3 * ulp / 2, -(1 + ulp / 2), 2 + 2 * ulp])  # the last is exact
+    got = bits_to_float(round_to_bf16_bits(ties))
+    assert got.tolist() == [1.0, 1 + 2 * ulp, -1.0, 2 + 2 * ulp]
+
+
+def test_rms_norm_of_a_constant_row_and_a_one_hot_row():
+    D = 128
+    x = np.zeros((1, 2, 1, D), np.float64)
+    x[0, 0, 0, :] = -3.0
+    x[0, 1, 0, 5] = 2.0
+    eps = 1e-6
+    y = rms_norm(to_bf16_bits(x), eps=eps)
+    assert np.allclose(y[0, 0, 0], -3.0 / math.sqrt(9.0 + eps), rtol=1e-15)
+    expect = np.zeros(D)
+    expect[5] = 2.0 / math.sqrt(4.0 / D + eps)      # = sqrt(D) as eps -> 0
+    assert np.allclose(y[0, 1, 0], expect, rtol=1e-15, atol=0)
+
+
+def test_rms_norm_output_has_unit_rms_and_ignores_power_of_two_scale():
+    g = torch.Generator().manual_seed(32)
+    x = (torch.randn(2, 9, 3, 128, generator=g, dtype=torch.float64) * 4).to(torch.bfloat16)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    y = rms_norm(xb, eps=0.0)
+    assert np.allclose(np.sqrt(np.mean(y * y, axis=-1)), 1.0, rtol=1e-13)
+    x8 = (x.double() * 8).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)  # exact in bf16
+    assert np.allclose(rms_norm(x8, eps=0.0), y, rtol=1e-13)
+
+
+def test_rms_norm_per_head_weight_matches_torch_rms_norm_head_by_head():
+    g = torch.Generator().manual_seed(33)
+    x = torch.randn(1, 17, 4, 128, generator=g, dtype=torch.float64).to(torch.bfloat16)
+    w = torch.rand(4, 128, generator=g, dtype=torch.float64) + 0.5
+    y = rms_norm(x.view(torch.int16).numpy().view(np.uint16), w.numpy(), eps=1e-6)
+    for h in range(4):
+        ref = torch.nn.functional.rms_norm(x[:, :, h].double(), (128,), weight=w[h], eps=1e-6)
+        assert np.allclose(y[:, :, h], ref.numpy(), rtol=1e-13, atol=1e-15)
+    with pytest.raises(ValueError):
+        rms_norm(x.view(torch.int16).numpy().view(np.uint16), w[:3].numpy())

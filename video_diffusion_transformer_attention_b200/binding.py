@@ -39,6 +39,9 @@ EXPORTS = (
     "vdit_attn_fwd_ws",
     "vdit_attn_fwd_block_sparse",
     "vdit_attn_merge",
+    "vdit_attn_fwd_qknorm",
+    "vdit_attn_qknorm_plan",
+    "vdit_qk_rms_norm",
     "vdit_get_device_status",
     "vdit_status_string",
     "vdit_abi_version",
@@ -78,6 +81,13 @@ def lib() -> ctypes.CDLL:
             h.vdit_attn_fwd_block_sparse.restype = c_int
             h.vdit_attn_fwd_block_sparse.argtypes = [vp, vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int,
                                                      c_float, vp]
+            h.vdit_attn_fwd_qknorm.restype = c_int
+            h.vdit_attn_fwd_qknorm.argtypes = [vp, vp, vp, vp, vp, vp, vp, c_float, c_int, c_int, c_int, c_int,
+                                               c_int, c_float, c_int, c_int, vp, c_size, vp]
+            h.vdit_attn_qknorm_plan.restype = c_int
+            h.vdit_attn_qknorm_plan.argtypes = [c_int] * 7 + [ctypes.POINTER(c_size)]
+            h.vdit_qk_rms_norm.restype = c_int
+            h.vdit_qk_rms_norm.argtypes = [vp, vp, vp, vp, vp, vp, c_float, c_int, c_int, c_int, c_int, c_int, vp]
             h.vdit_attn_merge.restype = c_int
             h.vdit_attn_merge.argtypes = [vp, vp, vp, vp, c_int, c_int, c_int, c_int, vp]
             h.vdit_testing_attn_fwd.restype = c_int
@@ -159,6 +169,34 @@ def vdit_attn_fwd_block_sparse(q, k, v, o, lse, block_mask, B, H, Sq, Skv, D, sc
     return st
 
 
+def vdit_qk_rms_norm(q, k, q_out, k_out, q_norm_weight, k_norm_weight, eps, B, H, Sq, Skv, D, stream=None,
+                     check=True) -> int:
+    """Per-head RMS norm of q and k into q_out, k_out (see include/vdit_attn.h)."""
+    st = lib().vdit_qk_rms_norm(_addr(q), _addr(k), _addr(q_out), _addr(k_out), _addr(q_norm_weight),
+                                _addr(k_norm_weight), float(eps), B, H, Sq, Skv, D, _stream(stream))
+    if check and st != VDIT_OK:
+        raise VditError(st, "vdit_qk_rms_norm")
+    return st
+
+
+def vdit_attn_qknorm_plan(B, H, Sq, Skv, D, mask_kind, chunk_tokens):
+    """Returns (status, workspace bytes) for vdit_attn_fwd_qknorm."""
+    ws = ctypes.c_size_t(0)
+    st = lib().vdit_attn_qknorm_plan(B, H, Sq, Skv, D, mask_kind, chunk_tokens, ctypes.byref(ws))
+    return int(st), int(ws.value)
+
+
+def vdit_attn_fwd_qknorm(q, k, v, o, lse, q_norm_weight, k_norm_weight, eps, B, H, Sq, Skv, D, scale, mask_kind,
+                         chunk_tokens, workspace, workspace_bytes, stream=None, check=True) -> int:
+    """Forward on raw Q/K: per-head RMS norm into the workspace, then attention (see include/vdit_attn.h)."""
+    st = lib().vdit_attn_fwd_qknorm(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), _addr(q_norm_weight),
+                                    _addr(k_norm_weight), float(eps), B, H, Sq, Skv, D, float(scale), mask_kind,
+                                    chunk_tokens, _addr(workspace), int(workspace_bytes), _stream(stream))
+    if check and st != VDIT_OK:
+        raise VditError(st, "vdit_attn_fwd_qknorm")
+    return st
+
+
 def vdit_attn_merge(o_acc, lse_acc, o_part, lse_part, B, H, S, D, stream=None, check=True) -> int:
     """Fold (o_part, lse_part) into (o_acc, lse_acc) in place (see include/vdit_attn.h)."""
     st = lib().vdit_attn_merge(_addr(o_acc), _addr(lse_acc), _addr(o_part), _addr(lse_part), B, H, S, D,
@@ -224,3 +262,36 @@ def attention_block_sparse(q, k, v, block_mask, scale=None, out=None, lse=None, 
         lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
     vdit_attn_fwd_block_sparse(q, k, v, out, lse, block_mask, B, H, Sq, Skv, D, scale, stream)
     return out, lse
+
+
+def attention_qknorm(q, k, v, q_norm_weight=None, k_norm_weight=None, eps=1e-6, scale=None,
+                     mask_kind=VDIT_MASK_FULL, chunk_tokens=0, workspace=None, stream=None):
+    """Convenience wrapper over vdit_attn_fwd_qknorm (raw CUDA bf16 q, k; fp32 [H, D] weights or None).
+
+    workspace: a CUDA uint8 tensor of at least vdit_attn_qknorm_plan bytes, or
+    None to allocate one with torch.  Returns (o, lse)."""
+    import torch
+    B, Sq, H, D = q.shape
+    Skv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / float(D) ** 0.5
+    st, need = vdit_attn_qknorm_plan(B, H, Sq, Skv, D, mask_kind, chunk_tokens)
+    if st != VDIT_OK:
+        raise VditError(st, "vdit_attn_qknorm_plan")
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    vdit_attn_fwd_qknorm(q, k, v, out, lse, q_norm_weight, k_norm_weight, eps, B, H, Sq, Skv, D, scale,
+                         mask_kind, chunk_tokens, workspace, workspace.numel(), stream)
+    return out, lse
+
+
+def qk_rms_norm(q, k, q_norm_weight=None, k_norm_weight=None, eps=1e-6, inplace=False, stream=None):
+    """Convenience wrapper over vdit_qk_rms_norm for CUDA bf16 [B, S, H, 128] q and k. Returns (q_n, k_n)."""
+    import torch
+    B, Sq, H, D = q.shape
+    Skv = k.shape[1]
+    q_out, k_out = (q, k) if inplace else (torch.empty_like(q), torch.empty_like(k))
+    vdit_qk_rms_norm(q, k, q_out, k_out, q_norm_weight, k_norm_weight, eps, B, H, Sq, Skv, D, stream)
+    return q_out, k_out

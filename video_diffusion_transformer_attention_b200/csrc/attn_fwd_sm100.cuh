@@ -305,6 +305,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         setmaxnreg_dec<kControlRegs>();
         if (warp == kLoadWarp && lane == 0) {
             // ------------------------------------------------ TMA producer
+            griddep_wait();  // Q/K written by a preceding kernel (fused Q/K norm) are complete
             for (int t = 0; n_kv > 0 && t < kQTiles; ++t) {
                 const uint32_t bar = smem_addr(&bars->q_full[t]);
                 mbar_arrive_expect_tx(bar, kTileBytes);

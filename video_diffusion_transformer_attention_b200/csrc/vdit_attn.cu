@@ -16,6 +16,7 @@
 #include "vdit_attn_testing.h"
 #include "attn_fwd_sm100.cuh"
 #include "attn_merge.cuh"
+#include "qk_norm.cuh"
 
 namespace {
 
@@ -57,6 +58,7 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 struct DeviceState {
     std::once_flag once;
     vdit_status status = VDIT_ERR_CUDA;
+    int norm_grid = 0;  // one full wave of qk_rms_norm_kernel blocks
 };
 DeviceState g_devices[kMaxDevices];
 
@@ -76,16 +78,26 @@ void init_device(int dev, DeviceState* st) {
         st->status = VDIT_ERR_CUDA;
         return;
     }
+    int sms = 0, per_sm = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, vdit::qk_rms_norm_kernel, vdit::kNormThreads, 0) !=
+            cudaSuccess ||
+        sms < 1 || per_sm < 1) {
+        st->status = VDIT_ERR_CUDA;
+        return;
+    }
+    st->norm_grid = sms * per_sm;
     st->status = VDIT_OK;
 }
 
-vdit_status ensure_device(int* dev_out) {
+vdit_status ensure_device(int* dev_out, const DeviceState** state_out = nullptr) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return VDIT_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return VDIT_ERR_UNSUPPORTED;
     DeviceState* st = &g_devices[dev];
     std::call_once(st->once, init_device, dev, st);
     *dev_out = dev;
+    if (state_out != nullptr) *state_out = st;
     return st->status;
 }
 
@@ -126,8 +138,8 @@ bool encode_bshd(CUtensorMap* map, const void* base, int B, int S, int H) {
 }
 
 vdit_status launch(const void* q, const void* k, const void* v, void* o, float* lse, const uint8_t* block_mask,
-                   const Shape& s, float scale, int debug_flags, unsigned long long timeout_ns,
-                   cudaStream_t stream) {
+                   const Shape& s, float scale, int debug_flags, unsigned long long timeout_ns, cudaStream_t stream,
+                   bool after_norm) {
     int dev = 0;
     vdit_status st = ensure_device(&dev);
     if (st != VDIT_OK) return st;
@@ -151,15 +163,32 @@ vdit_status launch(const void* q, const void* k, const void* v, void* o, float* 
     p.n_qb = (s.Sq + vdit::kSparseBlock - 1) / vdit::kSparseBlock;
     p.n_kvb = (s.Skv + vdit::kSparseBlock - 1) / vdit::kSparseBlock;
     dim3 grid(grid_x(s.Sq), s.H, s.B);
-    vdit::attn_fwd_sm100_kernel<<<grid, vdit::kNumThreads, vdit::kSmemBytes, stream>>>(tq, tk, tv, p);
-    return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
+    if (!after_norm) {
+        vdit::attn_fwd_sm100_kernel<<<grid, vdit::kNumThreads, vdit::kSmemBytes, stream>>>(tq, tk, tv, p);
+        return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
+    }
+    // Programmatic dependent of the Q/K norm kernel just queued on this
+    // stream: CTAs may start while it drains; the TMA producer waits for it
+    // (griddepcontrol.wait) before loading Q or K.
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(vdit::kNumThreads);
+    cfg.dynamicSmemBytes = vdit::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, vdit::attn_fwd_sm100_kernel, tq, tk, tv, p) == cudaSuccess ? VDIT_OK
+                                                                                             : VDIT_ERR_CUDA;
 }
 
 vdit_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
                      int Skv, int D, float scale, int mask_kind, int chunk_tokens, void* workspace,
                      size_t workspace_bytes, void* stream, int debug_flags = 0,
                      unsigned long long timeout_ns = kDefaultWaitTimeoutNs,
-                     const uint8_t* block_mask = nullptr) {
+                     const uint8_t* block_mask = nullptr, bool after_norm = false) {
     (void)workspace;
     (void)workspace_bytes;  // no shape needs a workspace in this version
     const Shape s{B, H, Sq, Skv, D, mask_kind, chunk_tokens};
@@ -188,8 +217,58 @@ vdit_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
             (lse != nullptr && overlaps(block_mask, mask_bytes, lse, size_t(B) * size_t(H) * size_t(Sq) * 4)))
             return VDIT_ERR_INVALID_ARG;
     }
-    return launch(q, k, v, o, lse, block_mask, s, scale, debug_flags, timeout_ns,
-                  static_cast<cudaStream_t>(stream));
+    return launch(q, k, v, o, lse, block_mask, s, scale, debug_flags, timeout_ns, static_cast<cudaStream_t>(stream),
+                  after_norm);
+}
+
+// ------------------------------------------------------------ Q/K RMS norm
+
+constexpr size_t kWorkspaceAlign = 256;
+
+size_t round_up(size_t n, size_t a) { return (n + a - 1) / a * a; }
+
+// Validates and queues the per-head RMS norm of q (B*Sq*H rows) and k
+// (B*Skv*H rows) into q_out / k_out.  Each output is the same address as its
+// input or disjoint from every input and output.
+vdit_status qk_norm_impl(const void* q, const void* k, void* q_out, void* k_out, const float* q_w, const float* k_w,
+                         float eps, int B, int H, int Sq, int Skv, int D, cudaStream_t stream) {
+    if (B < 0 || H < 0 || Sq < 0 || Skv < 0 || D < 1) return VDIT_ERR_INVALID_ARG;
+    if (D != vdit::kNormHeadDim) return VDIT_ERR_UNSUPPORTED;
+    if (!(std::isfinite(eps) && eps > 0.0f)) return VDIT_ERR_INVALID_ARG;
+    const long long q_rows = (long long)B * Sq * H, k_rows = (long long)B * Skv * H;
+    if (q_rows == 0 && k_rows == 0) return VDIT_OK;
+    if ((q_rows > 0 && (q == nullptr || q_out == nullptr)) || (k_rows > 0 && (k == nullptr || k_out == nullptr)))
+        return VDIT_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(q_out) || !aligned16(k_out) || !aligned16(q_w) ||
+        !aligned16(k_w))
+        return VDIT_ERR_MISALIGNED;
+    const size_t qb = size_t(q_rows) * 256, kb = size_t(k_rows) * 256;
+    const size_t wb = size_t(H) * vdit::kNormHeadDim * 4;
+    auto clash = [](const void* a, size_t na, const void* b, size_t nb) {  // overlap other than identity
+        return na > 0 && nb > 0 && a != b && overlaps(a, na, b, nb);
+    };
+    if (clash(q_out, qb, q, qb) || clash(k_out, kb, k, kb) || (qb > 0 && kb > 0 &&
+        (overlaps(q_out, qb, k, kb) || overlaps(k_out, kb, q, qb) || overlaps(q_out, qb, k_out, kb))))
+        return VDIT_ERR_INVALID_ARG;
+    if ((q_w != nullptr && ((qb > 0 && overlaps(q_w, wb, q_out, qb)) || (kb > 0 && overlaps(q_w, wb, k_out, kb)))) ||
+        (k_w != nullptr && ((qb > 0 && overlaps(k_w, wb, q_out, qb)) || (kb > 0 && overlaps(k_w, wb, k_out, kb)))))
+        return VDIT_ERR_INVALID_ARG;
+    int dev = 0;
+    const DeviceState* ds = nullptr;
+    const vdit_status st = ensure_device(&dev, &ds);
+    if (st != VDIT_OK) return st;
+    const long long passes = (q_rows + k_rows + 2 * vdit::kNormRowsInFlight - 1) / (2 * vdit::kNormRowsInFlight);
+    const long long want = (passes + vdit::kNormThreads / 32 - 1) / (vdit::kNormThreads / 32);
+    const unsigned grid = unsigned(want < ds->norm_grid ? want : ds->norm_grid);
+    const vdit::NormTensor a{static_cast<const uint4*>(q), static_cast<uint4*>(q_out), q_w, q_rows};
+    const vdit::NormTensor b{static_cast<const uint4*>(k), static_cast<uint4*>(k_out), k_w, k_rows};
+    vdit::qk_rms_norm_kernel<<<grid, vdit::kNormThreads, 0, stream>>>(a, b, H, eps);
+    return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
+}
+
+size_t qknorm_workspace_bytes(int B, int H, int Sq, int Skv, int D) {
+    const size_t row = size_t(H) * size_t(D) * 2;
+    return round_up(size_t(B) * size_t(Sq) * row, kWorkspaceAlign) + size_t(B) * size_t(Skv) * row;
 }
 
 }  // namespace
@@ -261,6 +340,68 @@ vdit_status vdit_attn_fwd_block_sparse(const void* q, const void* k, const void*
     }
 }
 
+vdit_status vdit_qk_rms_norm(const void* q, const void* k, void* q_out, void* k_out, const float* q_norm_weight,
+                             const float* k_norm_weight, float eps, int B, int H, int Sq, int Skv, int D,
+                             void* stream) {
+    try {
+        return qk_norm_impl(q, k, q_out, k_out, q_norm_weight, k_norm_weight, eps, B, H, Sq, Skv, D,
+                            static_cast<cudaStream_t>(stream));
+    } catch (...) {
+        return VDIT_ERR_CUDA;
+    }
+}
+
+vdit_status vdit_attn_qknorm_plan(int B, int H, int Sq, int Skv, int D, int mask_kind, int chunk_tokens,
+                                  size_t* workspace_bytes) {
+    try {
+        if (workspace_bytes == nullptr || mask_kind == VDIT_MASK_BLOCK_SPARSE) return VDIT_ERR_INVALID_ARG;
+        const Shape s{B, H, Sq, Skv, D, mask_kind, chunk_tokens};
+        const vdit_status st = check_shape(s, false, 1.0f);
+        if (st != VDIT_OK) return st;
+        *workspace_bytes = qknorm_workspace_bytes(B, H, Sq, Skv, D);
+        return VDIT_OK;
+    } catch (...) {
+        return VDIT_ERR_INVALID_ARG;
+    }
+}
+
+vdit_status vdit_attn_fwd_qknorm(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 const float* q_norm_weight, const float* k_norm_weight, float eps, int B, int H,
+                                 int Sq, int Skv, int D, float scale, int mask_kind, int chunk_tokens, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    try {
+        if (mask_kind == VDIT_MASK_BLOCK_SPARSE) return VDIT_ERR_INVALID_ARG;
+        const Shape s{B, H, Sq, Skv, D, mask_kind, chunk_tokens};
+        vdit_status st = check_shape(s, true, scale);
+        if (st != VDIT_OK) return st;
+        if (!(std::isfinite(eps) && eps > 0.0f)) return VDIT_ERR_INVALID_ARG;
+        if (!aligned16(q_norm_weight) || !aligned16(k_norm_weight)) return VDIT_ERR_MISALIGNED;
+        if (B == 0 || H == 0 || Sq == 0) return VDIT_OK;
+        const size_t need = qknorm_workspace_bytes(B, H, Sq, Skv, D);
+        if (workspace == nullptr || workspace_bytes < need) return VDIT_ERR_WORKSPACE;
+        if ((reinterpret_cast<uintptr_t>(workspace) & (kWorkspaceAlign - 1)) != 0) return VDIT_ERR_MISALIGNED;
+        const size_t row = size_t(H) * size_t(D) * 2;
+        const size_t qb = size_t(B) * size_t(Sq) * row, kb = size_t(B) * size_t(Skv) * row;
+        if (q == nullptr || k == nullptr || overlaps(workspace, need, q, qb) || overlaps(workspace, need, k, kb) ||
+            (v != nullptr && overlaps(workspace, need, v, kb)) ||
+            (lse != nullptr && overlaps(workspace, need, lse, size_t(B) * size_t(H) * size_t(Sq) * 4)))
+            return VDIT_ERR_INVALID_ARG;
+        void* q_n = workspace;
+        void* k_n = static_cast<char*>(workspace) + round_up(qb, kWorkspaceAlign);
+        if (v == nullptr || o == nullptr) return VDIT_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+            return VDIT_ERR_MISALIGNED;
+        if (overlaps(o, qb, q, qb) || overlaps(o, qb, k, kb)) return VDIT_ERR_INVALID_ARG;
+        st = qk_norm_impl(q, k, q_n, k_n, q_norm_weight, k_norm_weight, eps, B, H, Sq, Skv, D,
+                          static_cast<cudaStream_t>(stream));
+        if (st != VDIT_OK) return st;
+        return fwd_impl(q_n, k_n, v, o, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, nullptr, 0, stream, 0,
+                        kDefaultWaitTimeoutNs, nullptr, true);
+    } catch (...) {
+        return VDIT_ERR_CUDA;
+    }
+}
+
 vdit_status vdit_testing_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                                   int Sq, int Skv, int D, float scale, int mask_kind, int chunk_tokens,
                                   int fault, unsigned long long wait_timeout_ns, void* stream) {
@@ -294,8 +435,8 @@ vdit_status vdit_attn_merge(void* o_acc, float* lse_acc, const void* o_part, con
             overlaps(o_acc, o_bytes, lse_acc, l_bytes) || overlaps(o_acc, o_bytes, lse_part, l_bytes) ||
             overlaps(lse_acc, l_bytes, o_part, o_bytes))
             return VDIT_ERR_INVALID_ARG;
-        int sm_count = 0;
-        const vdit_status st = ensure_device(&sm_count);
+        int dev = 0;
+        const vdit_status st = ensure_device(&dev);
         if (st != VDIT_OK) return st;
         vdit::attn_merge_kernel<<<unsigned(blocks), vdit::kMergeWarpsPerBlock * 32, 0,
                                   static_cast<cudaStream_t>(stream)>>>(

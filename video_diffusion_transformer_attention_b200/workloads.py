@@ -116,14 +116,17 @@ def _scale_outlier_channels(v: torch.Tensor, gen: torch.Generator) -> torch.Tens
 
 
 def draw_qkv(B: int, H: int, Sq: int, Skv: int, D: int, seed: int,
-             recipe: str = "iid"):
-    """Draw bf16 (Q, K, V) on the CPU in [B, S, H, D] layout."""
+             recipe: str = "iid", raw_qk: bool = False):
+    """Draw bf16 (Q, K, V) on the CPU in [B, S, H, D] layout.
+
+    raw_qk: skip the RMS norm of Q and K that the recipe asks for (the fused
+    Q/K-norm entry point applies it inside the kernel instead)."""
     gen = torch.Generator(device="cpu")
     gen.manual_seed(int(seed))
     q = torch.randn((B, Sq, H, D), generator=gen, dtype=torch.float32)
     k = torch.randn((B, Skv, H, D), generator=gen, dtype=torch.float32)
     v = torch.randn((B, Skv, H, D), generator=gen, dtype=torch.float32)
-    if recipe in ("rms_qk", "rms_qk_vout"):
+    if recipe in ("rms_qk", "rms_qk_vout") and not raw_qk:
         q = _rms_normalise(q)
         k = _rms_normalise(k)
     if recipe == "rms_qk_vout":
@@ -142,7 +145,7 @@ def draw_text_kv(B: int, H: int, Skv: int, D: int, seed: int):
     return k.to(torch.bfloat16), v.to(torch.bfloat16)
 
 
-def workload_inputs(name: str):
+def workload_inputs(name: str, raw_qk: bool = False):
     """All inputs of a named workload, as a dict of CPU bf16 tensors.
 
     Keys: "q", "k", "v" (self-attention) and, for workloads with a text
@@ -151,7 +154,7 @@ def workload_inputs(name: str):
     w = WORKLOADS[name]
     self_call = w.calls[0]
     q, k, v = draw_qkv(self_call.B, self_call.H, self_call.Sq, self_call.Skv,
-                       self_call.D, 1000 + w.index, w.recipe)
+                       self_call.D, 1000 + w.index, w.recipe, raw_qk)
     out = {"q": q, "k": k, "v": v}
     if self_call.mask_kind == MASK_BLOCK_SPARSE:
         out["block_mask"] = draw_block_mask(self_call.B, self_call.H, self_call.Sq, self_call.Skv,
