@@ -187,6 +187,43 @@ vdit_status vdit_attn_fwd_qknorm(const void* q, const void* k, const void* v,
                                  void* stream);
 
 /*
+ * vdit_attn_fwd_qknorm_noalloc -- vdit_attn_fwd_qknorm for callers that
+ * cannot allocate device memory: the normalised Q and K go to a scratch
+ * buffer built into the library (VDIT_NOALLOC_SCRATCH_BYTES, a fixed
+ * device-memory array that every GPU loading the library holds until the
+ * process exits) instead of a workspace passed in.  The pages this library
+ * follows have no counterpart of this entry point.
+ *
+ * It exists for code that must not call cudaMalloc: a plugin inside a host
+ * application that owns all of the GPU's memory through its own pool (a raw
+ * cudaMalloc there bypasses the pool's accounting and can fail once the pool
+ * has reserved the rest of the device), and latency-critical loops where
+ * cudaMalloc / cudaFree may synchronise the device and stall other work.
+ * The entry point itself calls neither.
+ *
+ * Arguments, layouts and results are those of vdit_attn_fwd_qknorm, minus
+ * the workspace.  Shapes whose normalised Q and K need more than
+ * VDIT_NOALLOC_SCRATCH_BYTES (vdit_attn_qknorm_plan gives the need) return
+ * VDIT_ERR_WORKSPACE with nothing launched.
+ *
+ * The first call on a device looks up the scratch's device address (once
+ * per device, with that device current); make that first call before any
+ * stream capture.  All calls on a device share the one scratch buffer and it
+ * keeps the last call's contents (nothing in it needs to start at zero), so
+ * calls whose work overlaps on the GPU (other streams, or other host threads
+ * without ordering between their streams) race on it: order them.
+ */
+#define VDIT_NOALLOC_SCRATCH_BYTES (64u << 20) /* 64 MiB */
+
+vdit_status vdit_attn_fwd_qknorm_noalloc(const void* q, const void* k,
+                                         const void* v, void* o, float* lse,
+                                         const float* q_norm_weight,
+                                         const float* k_norm_weight, float eps,
+                                         int B, int H, int Sq, int Skv, int D,
+                                         float scale, int mask_kind,
+                                         int chunk_tokens, void* stream);
+
+/*
  * vdit_attn_fwd_ws -- vdit_attn_fwd with a caller-owned device workspace of
  * `workspace_bytes` bytes (at least what vdit_attn_plan reports; NULL is
  * accepted when that is 0).

@@ -42,6 +42,7 @@ EXPORTS = (
     "vdit_attn_fwd_qknorm",
     "vdit_attn_qknorm_plan",
     "vdit_qk_rms_norm",
+    "vdit_attn_fwd_qknorm_noalloc",
     "vdit_get_device_status",
     "vdit_status_string",
     "vdit_abi_version",
@@ -86,6 +87,9 @@ def lib() -> ctypes.CDLL:
                                                c_int, c_float, c_int, c_int, vp, c_size, vp]
             h.vdit_attn_qknorm_plan.restype = c_int
             h.vdit_attn_qknorm_plan.argtypes = [c_int] * 7 + [ctypes.POINTER(c_size)]
+            h.vdit_attn_fwd_qknorm_noalloc.restype = c_int
+            h.vdit_attn_fwd_qknorm_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, c_float, c_int, c_int, c_int,
+                                                       c_int, c_int, c_float, c_int, c_int, vp]
             h.vdit_qk_rms_norm.restype = c_int
             h.vdit_qk_rms_norm.argtypes = [vp, vp, vp, vp, vp, vp, c_float, c_int, c_int, c_int, c_int, c_int, vp]
             h.vdit_attn_merge.restype = c_int
@@ -194,6 +198,21 @@ def vdit_attn_fwd_qknorm(q, k, v, o, lse, q_norm_weight, k_norm_weight, eps, B, 
                                     chunk_tokens, _addr(workspace), int(workspace_bytes), _stream(stream))
     if check and st != VDIT_OK:
         raise VditError(st, "vdit_attn_fwd_qknorm")
+    return st
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20  # VDIT_NOALLOC_SCRATCH_BYTES in include/vdit_attn.h
+
+
+def vdit_attn_fwd_qknorm_noalloc(q, k, v, o, lse, q_norm_weight, k_norm_weight, eps, B, H, Sq, Skv, D, scale,
+                                 mask_kind, chunk_tokens, stream=None, check=True) -> int:
+    """vdit_attn_fwd_qknorm without a workspace argument: the library's fixed device scratch holds the
+    normalised Q and K, so nothing is allocated (see include/vdit_attn.h)."""
+    st = lib().vdit_attn_fwd_qknorm_noalloc(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse),
+                                            _addr(q_norm_weight), _addr(k_norm_weight), float(eps), B, H, Sq, Skv,
+                                            D, float(scale), mask_kind, chunk_tokens, _stream(stream))
+    if check and st != VDIT_OK:
+        raise VditError(st, "vdit_attn_fwd_qknorm_noalloc")
     return st
 
 

@@ -273,6 +273,33 @@ size_t qknorm_workspace_bytes(int B, int H, int Sq, int Skv, int D) {
 
 }  // namespace
 
+// ------------------------------------------------------------ fixed scratch, no allocation
+//
+// Backing store of vdit_attn_fwd_qknorm_noalloc: the normalised Q and K live
+// here instead of in a caller workspace.  Every GPU that loads the library
+// holds these bytes until the process exits.  Host code must not pass the
+// array's name to a kernel (on the host it is only a stand-in symbol); the
+// device address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[VDIT_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+struct NoAllocScratch {
+    std::once_flag once;
+    cudaError_t err = cudaErrorUnknown;
+    void* ptr = nullptr;
+};
+NoAllocScratch g_noalloc[kMaxDevices];
+
+// Called with `dev` current (the entry point runs it for the current device).
+void resolve_noalloc_scratch(NoAllocScratch* st) {
+    void* p = nullptr;
+    st->err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    st->ptr = st->err == cudaSuccess ? p : nullptr;
+}
+
+}  // namespace
+
 extern "C" {
 
 int vdit_abi_version(void) { return VDIT_ATTN_ABI_VERSION; }
@@ -397,6 +424,33 @@ vdit_status vdit_attn_fwd_qknorm(const void* q, const void* k, const void* v, vo
         if (st != VDIT_OK) return st;
         return fwd_impl(q_n, k_n, v, o, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, nullptr, 0, stream, 0,
                         kDefaultWaitTimeoutNs, nullptr, true);
+    } catch (...) {
+        return VDIT_ERR_CUDA;
+    }
+}
+
+vdit_status vdit_attn_fwd_qknorm_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                                         const float* q_norm_weight, const float* k_norm_weight, float eps, int B,
+                                         int H, int Sq, int Skv, int D, float scale, int mask_kind,
+                                         int chunk_tokens, void* stream) {
+    try {
+        if (mask_kind == VDIT_MASK_BLOCK_SPARSE) return VDIT_ERR_INVALID_ARG;
+        const Shape s{B, H, Sq, Skv, D, mask_kind, chunk_tokens};
+        const vdit_status st = check_shape(s, true, scale);
+        if (st != VDIT_OK) return st;
+        if (B == 0 || H == 0 || Sq == 0) return VDIT_OK;
+        if (qknorm_workspace_bytes(B, H, Sq, Skv, D) > size_t(VDIT_NOALLOC_SCRATCH_BYTES))
+            return VDIT_ERR_WORKSPACE;  // the shape does not fit the fixed scratch
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return VDIT_ERR_CUDA;
+        if (dev < 0 || dev >= kMaxDevices) return VDIT_ERR_UNSUPPORTED;
+        NoAllocScratch* sc = &g_noalloc[dev];
+        std::call_once(sc->once, resolve_noalloc_scratch, sc);
+        if (sc->err != cudaSuccess || sc->ptr == nullptr) return VDIT_ERR_CUDA;
+        // Nothing in the scratch has to start at zero: the norm writes all of
+        // the normalised Q and K before the attention reads them.
+        return vdit_attn_fwd_qknorm(q, k, v, o, lse, q_norm_weight, k_norm_weight, eps, B, H, Sq, Skv, D, scale,
+                                    mask_kind, chunk_tokens, sc->ptr, size_t(VDIT_NOALLOC_SCRATCH_BYTES), stream);
     } catch (...) {
         return VDIT_ERR_CUDA;
     }
