@@ -270,9 +270,27 @@ def run_vdit(args):
         if st != vb.VDIT_OK:
             raise SystemExit(f"vdit_attn_qknorm_plan: {vb.vdit_status_string(st)}")
         qk_ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    fp8_ws = []
+    if args.path == "fp8":
+        for c in w.calls:
+            st, need = vb.vdit_attn_fp8_plan(c.B, c.H, c.Sq, c.Skv, c.D, c.mask_kind, c.chunk_tokens)
+            if st != vb.VDIT_OK:
+                raise SystemExit(f"vdit_attn_fp8_plan: {vb.vdit_status_string(st)}")
+            fp8_ws.append(torch.empty(need, dtype=torch.uint8, device=dev))
+    # kernels this library launches per call of the step
+    launches_per_call = [(5 if args.path == "fp8" else 1) + (1 if args.qknorm and c.name == "self" else 0)
+                         for c in w.calls]
 
-    def launch(i, call, q, k, v, o, lse):
-        if args.qknorm and call.name == "self":
+    def launch(i, call, q, k, v, o, lse, mid_event=None):
+        if args.path == "fp8":
+            # quantise (one memset + three kernels), then the 8-bit attention
+            ws = fp8_ws[i]
+            vb.vdit_fp8_quantize(q, k, v, call.B, call.H, call.Sq, call.Skv, call.D, ws, ws.numel(), sptr)
+            if mid_event is not None:
+                mid_event.record(stream)
+            vb.vdit_attn_fwd_fp8_quantized(o, lse, call.B, call.H, call.Sq, call.Skv, call.D, call.scale,
+                                           call.mask_kind, call.chunk_tokens, ws, ws.numel(), sptr)
+        elif args.qknorm and call.name == "self":
             vb.vdit_attn_fwd_qknorm(q, k, v, o, lse, None, None, wl.RMS_EPS, call.B, call.H, call.Sq, call.Skv,
                                     call.D, call.scale, call.mask_kind, call.chunk_tokens, qk_ws, qk_ws.numel(),
                                     sptr)
@@ -288,7 +306,7 @@ def run_vdit(args):
             q, k, v = call_inputs(inp, call)
             if events is not None:
                 events[i][0].record(stream)
-            launch(i, call, q, k, v, *outs[i])
+            launch(i, call, q, k, v, *outs[i], mid_event=events[i][2] if events is not None else None)
             if events is not None:
                 events[i][1].record(stream)
 
@@ -300,7 +318,7 @@ def run_vdit(args):
     if st != vb.VDIT_OK:
         raise SystemExit(f"device status after warm-up: {vb.vdit_status_string(st)} ({word:#x})")
 
-    per_call_events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    per_call_events = [[tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
                         for _ in w.calls] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local_rank)
@@ -319,6 +337,11 @@ def run_vdit(args):
     ms = t_start.elapsed_time(t_end)
     call_ms = [statistics.mean(per_call_events[s][i][0].elapsed_time(per_call_events[s][i][1])
                                for s in range(args.steps)) for i in range(len(w.calls))]
+    # the attention kernel alone (8-bit path: after the quantisation launches)
+    kernel_ms = list(call_ms)
+    if args.path == "fp8":
+        kernel_ms = [statistics.mean(per_call_events[s][i][2].elapsed_time(per_call_events[s][i][1])
+                                     for s in range(args.steps)) for i in range(len(w.calls))]
     st, word = vb.vdit_get_device_status(sptr)
     if st != vb.VDIT_OK:
         raise SystemExit(f"device status after timing: {vb.vdit_status_string(st)} ({word:#x})")
@@ -364,34 +387,44 @@ def run_vdit(args):
         peaks, peak_src = load_peaks()
         # the self-attention launch dominates the step
         dom = 0
-        achieved = flops_per_call[dom] / (call_ms[dom] * 1e-3) / 1e12
-        peak_sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-        peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        achieved = flops_per_call[dom] / (kernel_ms[dom] * 1e-3) / 1e12
+        # an E4M3 contraction takes twice the bf16 peak (nominal 4.5 vs 2.25 PFLOP/s dense)
+        dtype_ratio = 2.0 if args.path == "fp8" else 1.0
+        peak_sustained = dtype_ratio * float(peaks.get("bf16_tflops_sustained",
+                                                       FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        peak_burst = dtype_ratio * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
         cross = w.calls[1] if len(w.calls) > 1 else None
         calls = []
         for i, c in enumerate(w.calls):
             calls.append({"call": c.name, "ms": call_ms[i], "tflops": flops_per_call[i] / (call_ms[i] * 1e-3) / 1e12,
                           "hbm_gbs": fl.attn_min_bytes(c) / (call_ms[i] * 1e-3) / 1e9})
+            if args.path == "fp8":
+                calls[-1]["attention_kernel_ms"] = kernel_ms[i]
+                calls[-1]["quantize_ms"] = call_ms[i] - kernel_ms[i]
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": "e4m3" if args.path == "fp8" else "bf16", "data": "synthetic",
             "config": {"workload": f"{args.workload} ({desc})" + (" [raw Q/K: per-head RMS norm + attention]"
-                                                                  if args.qknorm else ""),
+                                                                  if args.qknorm else "")
+                       + (" [8-bit path: E4M3 + V-Smooth + ExpCast-FP8, quantisation inside the step]"
+                          if args.path == "fp8" else ""),
                        "l2": "inputs larger than L2 (3.1 GB per step)",
                        "parallelism": f"independent replicas x{world} (no collective)"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_sustained, "unit": "TFLOP/s",
                          "frac": achieved / peak_sustained,
-                         "traffic": recorded_traffic() if args.workload == WORKLOAD else None,
-                         "kernel": "attn_fwd_sm100_kernel (self-attention launch)" if not args.qknorm else
-                                   "qk_rms_norm_kernel + attn_fwd_sm100_kernel (self-attention call)",
-                         "peak_kind": f"{peak_src} sustained bf16 (cuBLAS, power-capped)",
+                         "traffic": recorded_traffic() if args.workload == WORKLOAD and args.path == "bf16" else None,
+                         "kernel": ("attn_fwd_fp8_sm100_kernel (self-attention launch)" if args.path == "fp8" else
+                                    "attn_fwd_sm100_kernel (self-attention launch)" if not args.qknorm else
+                                    "qk_rms_norm_kernel + attn_fwd_sm100_kernel (self-attention call)"),
+                         "peak_kind": (f"{peak_src} sustained bf16 (cuBLAS, power-capped)" if args.path == "bf16" else
+                                       f"2 x {peak_src} sustained bf16 (E4M3 at the nominal 2:1 ratio)"),
                          "frac_of_burst": achieved / peak_burst,
                          "frac_of_datasheet": achieved / DATASHEET_BF16_TFLOPS},
             "calls": calls,
             "clocks": clk,
             "e2e": e2e,
-            "gpu_launches": len(w.calls) * args.steps,
+            "gpu_launches": sum(launches_per_call) * args.steps,
         }
         if cross is not None:
             line["roofline"]["cross_hbm_frac"] = calls[1]["hbm_gbs"] / float(peaks.get("hbm_gbs", 6650.0))
@@ -452,11 +485,15 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--reference-seconds", type=float, default=40.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", choices=("bf16", "fp8"), default="bf16",
+                    help="bf16 attention (default) or the 8-bit path (E4M3 + V-Smooth + ExpCast-FP8)")
     ap.add_argument("--qknorm", action="store_true",
                     help="raw Q/K with the per-head RMS norm fused into the self-attention call")
     ap.add_argument("--kernel", choices=("attention", "merge"), default="attention",
                     help="merge: time only the LSE merge kernel (HBM roofline)")
     args = ap.parse_args()
+    if args.path == "fp8" and args.qknorm:
+        ap.error("--qknorm applies to the bf16 path only")
     if args.warmup < 3 and args.impl == "vdit":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":

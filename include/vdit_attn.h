@@ -224,6 +224,71 @@ vdit_status vdit_attn_fwd_qknorm_noalloc(const void* q, const void* k,
                                          int chunk_tokens, void* stream);
 
 /*
+ * 8-bit path: "VC-Attention: revolution in video generation speed without
+ * retraining" (aikraft.ru), sections 02 (V-Smooth) and 03 (ExpCast-FP8).
+ *
+ *  - Q and K become E4M3 codes per 128-token block of one (b, h), scale =
+ *    block absmax / 448.
+ *  - V-Smooth: per 128-token block the mean is subtracted; the residual is
+ *    quantised to E4M3 with one scale per (b, h, channel) = max(max |residual|,
+ *    2^-8 max |block mean|) / 448; the block mean is added back through the
+ *    softmax row sum.
+ *  - ExpCast-FP8: each probability's E4M3 byte is written from the
+ *    log-domain score as rint(8 log2(p 2^5) + 56 - 0.35) with one FMA, no
+ *    exponential; the reference maximum is kept on the grid N + 0.65 (code
+ *    units, 8 x log2) and raised only when a tile's max exceeds it by more
+ *    than 24 codes.
+ * O is bf16 and LSE fp32 as in vdit_attn_fwd; the result differs from
+ * vdit_attn_fwd by the 8-bit quantisation (a few percent relative RMS on
+ * iid data).  Masks: FULL, BLOCK_CAUSAL, CROSS.  D must be 128.
+ *
+ * The caller owns a device workspace (256-byte aligned, size from
+ * vdit_attn_fp8_plan) that holds the codes; its parts, in this order, are
+ * located by vdit_fp8_layout:
+ */
+enum {
+    VDIT_FP8_PART_Q = 0,       /* uint8 [B][Sq][H][128]  E4M3 codes of Q        */
+    VDIT_FP8_PART_K = 1,       /* uint8 [B][Skv][H][128] E4M3 codes of K        */
+    VDIT_FP8_PART_VT = 2,      /* uint8 [B][H][nkb][128 ch][128 tok] V residual codes, per block transposed */
+    VDIT_FP8_PART_MU_IMG = 3,  /* [B][H][nkb] 4 KB restore tiles (bf16 block mean / channel scale, hi/lo) */
+    VDIT_FP8_PART_Q_SCALE = 4, /* fp32 [B][H][nqb]                            */
+    VDIT_FP8_PART_K_SCALE = 5, /* fp32 [B][H][nkb]                            */
+    VDIT_FP8_PART_V_SCALE = 6, /* fp32 [B][H][128]                            */
+    VDIT_FP8_PART_V_AMAX = 7,  /* scratch of the V statistics                 */
+    VDIT_FP8_PART_MU = 8,      /* fp32 [B][H][nkb][128] block means of V      */
+    VDIT_FP8_NUM_PARTS = 9
+};
+
+/* Host-only: offsets[0..8] = byte offset of each part, offsets[9] = total. */
+vdit_status vdit_fp8_layout(int B, int H, int Sq, int Skv, int D, size_t* offsets);
+
+/* Host-only: workspace bytes of the 8-bit path for this shape. */
+vdit_status vdit_attn_fp8_plan(int B, int H, int Sq, int Skv, int D,
+                               int mask_kind, int chunk_tokens,
+                               size_t* workspace_bytes);
+
+/* Quantise bf16 q, k, v into the workspace (four launches on `stream`). */
+vdit_status vdit_fp8_quantize(const void* q, const void* k, const void* v,
+                              int B, int H, int Sq, int Skv, int D,
+                              void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/* The 8-bit attention on a workspace that vdit_fp8_quantize filled. */
+vdit_status vdit_attn_fwd_fp8_quantized(void* o, float* lse, int B, int H,
+                                        int Sq, int Skv, int D, float scale,
+                                        int mask_kind, int chunk_tokens,
+                                        const void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
+/* vdit_fp8_quantize, then the 8-bit attention as a programmatic dependent
+ * launch.  Errors as vdit_attn_fwd, plus VDIT_ERR_WORKSPACE. */
+vdit_status vdit_attn_fwd_fp8(const void* q, const void* k, const void* v,
+                              void* o, float* lse, int B, int H, int Sq,
+                              int Skv, int D, float scale, int mask_kind,
+                              int chunk_tokens, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/*
  * vdit_attn_fwd_ws -- vdit_attn_fwd with a caller-owned device workspace of
  * `workspace_bytes` bytes (at least what vdit_attn_plan reports; NULL is
  * accepted when that is 0).

@@ -43,6 +43,11 @@ EXPORTS = (
     "vdit_attn_qknorm_plan",
     "vdit_qk_rms_norm",
     "vdit_attn_fwd_qknorm_noalloc",
+    "vdit_fp8_layout",
+    "vdit_attn_fp8_plan",
+    "vdit_fp8_quantize",
+    "vdit_attn_fwd_fp8_quantized",
+    "vdit_attn_fwd_fp8",
     "vdit_get_device_status",
     "vdit_status_string",
     "vdit_abi_version",
@@ -90,6 +95,16 @@ def lib() -> ctypes.CDLL:
             h.vdit_attn_fwd_qknorm_noalloc.restype = c_int
             h.vdit_attn_fwd_qknorm_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, c_float, c_int, c_int, c_int,
                                                        c_int, c_int, c_float, c_int, c_int, vp]
+            h.vdit_fp8_layout.restype = c_int
+            h.vdit_fp8_layout.argtypes = [c_int] * 5 + [ctypes.POINTER(c_size)]
+            h.vdit_attn_fp8_plan.restype = c_int
+            h.vdit_attn_fp8_plan.argtypes = [c_int] * 7 + [ctypes.POINTER(c_size)]
+            h.vdit_fp8_quantize.restype = c_int
+            h.vdit_fp8_quantize.argtypes = [vp, vp, vp] + [c_int] * 5 + [vp, c_size, vp]
+            h.vdit_attn_fwd_fp8_quantized.restype = c_int
+            h.vdit_attn_fwd_fp8_quantized.argtypes = [vp, vp] + [c_int] * 5 + [c_float, c_int, c_int, vp, c_size, vp]
+            h.vdit_attn_fwd_fp8.restype = c_int
+            h.vdit_attn_fwd_fp8.argtypes = fwd_args + [vp, c_size, vp]
             h.vdit_qk_rms_norm.restype = c_int
             h.vdit_qk_rms_norm.argtypes = [vp, vp, vp, vp, vp, vp, c_float, c_int, c_int, c_int, c_int, c_int, vp]
             h.vdit_attn_merge.restype = c_int
@@ -199,6 +214,72 @@ def vdit_attn_fwd_qknorm(q, k, v, o, lse, q_norm_weight, k_norm_weight, eps, B, 
     if check and st != VDIT_OK:
         raise VditError(st, "vdit_attn_fwd_qknorm")
     return st
+
+
+FP8_PARTS = ("q", "k", "vt", "mu_img", "q_scale", "k_scale", "v_scale", "v_amax", "mu")
+
+
+def vdit_fp8_layout(B, H, Sq, Skv, D):
+    """Returns (status, {part: byte offset}, total bytes) of the 8-bit path's workspace."""
+    off = (ctypes.c_size_t * (len(FP8_PARTS) + 1))()
+    st = lib().vdit_fp8_layout(B, H, Sq, Skv, D, off)
+    return int(st), dict(zip(FP8_PARTS, [int(x) for x in off[:-1]])), int(off[len(FP8_PARTS)])
+
+
+def vdit_attn_fp8_plan(B, H, Sq, Skv, D, mask_kind, chunk_tokens):
+    """Returns (status, workspace bytes) of the 8-bit path."""
+    ws = ctypes.c_size_t(0)
+    st = lib().vdit_attn_fp8_plan(B, H, Sq, Skv, D, mask_kind, chunk_tokens, ctypes.byref(ws))
+    return int(st), int(ws.value)
+
+
+def vdit_fp8_quantize(q, k, v, B, H, Sq, Skv, D, workspace, workspace_bytes, stream=None, check=True) -> int:
+    st = lib().vdit_fp8_quantize(_addr(q), _addr(k), _addr(v), B, H, Sq, Skv, D, _addr(workspace),
+                                 int(workspace_bytes), _stream(stream))
+    if check and st != VDIT_OK:
+        raise VditError(st, "vdit_fp8_quantize")
+    return st
+
+
+def vdit_attn_fwd_fp8_quantized(o, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, workspace,
+                                workspace_bytes, stream=None, check=True) -> int:
+    st = lib().vdit_attn_fwd_fp8_quantized(_addr(o), _addr(lse), B, H, Sq, Skv, D, float(scale), mask_kind,
+                                           chunk_tokens, _addr(workspace), int(workspace_bytes), _stream(stream))
+    if check and st != VDIT_OK:
+        raise VditError(st, "vdit_attn_fwd_fp8_quantized")
+    return st
+
+
+def vdit_attn_fwd_fp8(q, k, v, o, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, workspace,
+                      workspace_bytes, stream=None, check=True) -> int:
+    st = lib().vdit_attn_fwd_fp8(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), B, H, Sq, Skv, D,
+                                 float(scale), mask_kind, chunk_tokens, _addr(workspace), int(workspace_bytes),
+                                 _stream(stream))
+    if check and st != VDIT_OK:
+        raise VditError(st, "vdit_attn_fwd_fp8")
+    return st
+
+
+def attention_fp8(q, k, v, scale=None, mask_kind=VDIT_MASK_FULL, chunk_tokens=0, workspace=None, stream=None):
+    """Convenience wrapper over vdit_attn_fwd_fp8 for CUDA bf16 [B, S, H, 128] tensors.
+
+    workspace: a CUDA uint8 tensor of at least vdit_attn_fp8_plan bytes, or None
+    to allocate one with torch.  Returns (o, lse, workspace)."""
+    import torch
+    B, Sq, H, D = q.shape
+    Skv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / float(D) ** 0.5
+    st, need = vdit_attn_fp8_plan(B, H, Sq, Skv, D, mask_kind, chunk_tokens)
+    if st != VDIT_OK:
+        raise VditError(st, "vdit_attn_fp8_plan")
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    vdit_attn_fwd_fp8(q, k, v, out, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, workspace,
+                      workspace.numel(), stream)
+    return out, lse, workspace
 
 
 NOALLOC_SCRATCH_BYTES = 64 << 20  # VDIT_NOALLOC_SCRATCH_BYTES in include/vdit_attn.h

@@ -1,0 +1,203 @@
+// fp8_quant.cuh -- preprocessing of the 8-bit attention path: E4M3 codes of
+// Q and K per 128-token block, and V-Smooth for V.
+//
+// "VC-Attention: revolution in video generation speed without retraining"
+// (aikraft.ru), section 02 "V-Smooth": per hardware block of 128 tokens the
+// mean of V is subtracted ("Demean") and only the residual is quantised per
+// channel to E4M3; the mean goes back in through the softmax row sum
+// ("Restore").  Section 04: the preprocessing is fused into few kernels.
+//
+// Workspace contents written here (byte offsets from Fp8Layout):
+//   q8, k8    E4M3 codes, [B][S][H][128], the layout of Q and K
+//   vt8       E4M3 residual codes of V, per block transposed:
+//             [B][H][nkb][128 channels][128 tokens] (the K-major B operand of P.V)
+//   mu_img    per block, the 4 KB shared-memory image of the restore operand:
+//             a 16 x 128 bf16 tile, MN-major, 128B-swizzled, two 64-channel
+//             halves of 16 rows x 128 B; rows 0, 1, 2 hold mu'_hi, mu'_hi,
+//             mu'_lo (mu' = block mean in units of the channel scale), the
+//             other rows are zero
+//   q_scale, k_scale   fp32 [B][H][nb]: amax / 448 per block
+//   v_scale   fp32 [B][H][128]: per channel of a head, amax / 448
+//   v_amax_r, v_amax_mu  uint32 [B][H][128]: running maxima (fp32 bits) of
+//             |residual| and |block mean| over the head's blocks; zeroed by
+//             the host before v_stats_kernel
+//   mu        fp32 [B][H][nkb][128]: block means
+//
+// Every quantity that decides a stored code is computed with the same fp32
+// operations in the same order as the test oracle: amax exactly, the
+// quotients 448 / amax and amax / 448 with IEEE division, products rounded
+// to fp32, the block mean as a sequential fp32 sum divided by the token
+// count, and the E4M3 conversion rounding to nearest even with saturation.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cstdint>
+
+namespace vdit {
+
+constexpr int kQuantBlock = 128;          // tokens per block
+constexpr float kE4M3Max = 448.0f;
+constexpr float kMuFloor = 1.0f / 256.0f;  // channel amax >= 2^-8 x max |block mean|
+constexpr int kMuImgBytes = 4096;
+
+struct Fp8Tensors {
+    uint8_t* q8;
+    uint8_t* k8;
+    uint8_t* vt8;
+    uint8_t* mu_img;
+    float* q_scale;
+    float* k_scale;
+    float* v_scale;
+    uint32_t* v_amax_r;
+    uint32_t* v_amax_mu;
+    float* mu;
+};
+
+// Two fp32 values -> two E4M3 codes (low byte = a), nearest even, saturating.
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+    return uint32_t(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
+}
+
+// One CTA (128 threads) per (tensor, b, h, block).  Warp w holds tokens
+// 32w .. 32w+31 of the block; lane l holds channels 4l .. 4l+3 of each, so
+// every load and store instruction of a warp covers one whole token row.
+__global__ void __launch_bounds__(128)
+    qk_quant_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, Fp8Tensors t,
+                    int B, int H, int Sq, int Skv) {
+    __shared__ float warp_max[4];
+    const int nqb = (Sq + kQuantBlock - 1) / kQuantBlock;
+    const int nkb = (Skv + kQuantBlock - 1) / kQuantBlock;
+    long long id = blockIdx.x;
+    const long long n_q = static_cast<long long>(B) * H * nqb;
+    const bool is_k = id >= n_q;
+    if (is_k) id -= n_q;
+    const int nb = is_k ? nkb : nqb;
+    const int S = is_k ? Skv : Sq;
+    const int blk = static_cast<int>(id % nb);
+    const int h = static_cast<int>((id / nb) % H);
+    const int b = static_cast<int>(id / (static_cast<long long>(nb) * H));
+    const __nv_bfloat16* src = is_k ? k : q;
+    uint8_t* dst = is_k ? t.k8 : t.q8;
+    float* scale_out = is_k ? t.k_scale : t.q_scale;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tok0 = blk * kQuantBlock + warp * 32;
+    uint2 x[32];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int tok = tok0 + i;
+        x[i] = make_uint2(0u, 0u);
+        if (tok < S)
+            x[i] = *reinterpret_cast<const uint2*>(src + ((static_cast<size_t>(b) * S + tok) * H + h) * 128 + lane * 4);
+        const __nv_bfloat162* v = reinterpret_cast<const __nv_bfloat162*>(&x[i]);
+        const float2 f0 = __bfloat1622float2(v[0]), f1 = __bfloat1622float2(v[1]);
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(f0.x), fabsf(f0.y)), fmaxf(fabsf(f1.x), fabsf(f1.y))));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (lane == 0) warp_max[warp] = amax;
+    __syncthreads();
+    amax = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
+    const float inv = amax > 0.0f ? kE4M3Max / amax : 0.0f;
+    if (threadIdx.x == 0) scale_out[(static_cast<size_t>(b) * H + h) * nb + blk] = amax / kE4M3Max;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int tok = tok0 + i;
+        if (tok >= S) break;
+        const __nv_bfloat162* v = reinterpret_cast<const __nv_bfloat162*>(&x[i]);
+        const float2 f0 = __bfloat1622float2(v[0]), f1 = __bfloat1622float2(v[1]);
+        const uint32_t c = e4m3x2(f0.x * inv, f0.y * inv) | (e4m3x2(f1.x * inv, f1.y * inv) << 16);
+        *reinterpret_cast<uint32_t*>(dst + ((static_cast<size_t>(b) * S + tok) * H + h) * 128 + lane * 4) = c;
+    }
+}
+
+// One CTA (128 threads) per (b, h, block); thread d owns channel d.
+// Block mean (sequential fp32 sum over the block's tokens, then / n), the
+// block's largest |v - mean|, and the running per-channel maxima over the
+// head's blocks (atomicMax on the bits of non-negative floats, which order
+// like the floats).
+__global__ void __launch_bounds__(128)
+    v_stats_kernel(const __nv_bfloat16* __restrict__ v, Fp8Tensors t, int B, int H, int Skv) {
+    const int nkb = (Skv + kQuantBlock - 1) / kQuantBlock;
+    const int blk = blockIdx.x % nkb;
+    const int h = (blockIdx.x / nkb) % H;
+    const int b = blockIdx.x / (nkb * H);
+    const int d = threadIdx.x;
+    const int t0 = blk * kQuantBlock;
+    const int n = min(kQuantBlock, Skv - t0);
+    const __nv_bfloat16* col = v + ((static_cast<size_t>(b) * Skv + t0) * H + h) * 128 + d;
+    const size_t stride = static_cast<size_t>(H) * 128;
+    float sum = 0.0f;
+#pragma unroll 16
+    for (int i = 0; i < n; ++i) sum += __bfloat162float(col[i * stride]);
+    const float mu = sum / static_cast<float>(n);
+    float rmax = 0.0f;
+#pragma unroll 16
+    for (int i = 0; i < n; ++i) rmax = fmaxf(rmax, fabsf(__bfloat162float(col[i * stride]) - mu));
+    const size_t bh = static_cast<size_t>(b) * H + h;
+    t.mu[(bh * nkb + blk) * 128 + d] = mu;
+    atomicMax(t.v_amax_r + bh * 128 + d, __float_as_uint(rmax));
+    atomicMax(t.v_amax_mu + bh * 128 + d, __float_as_uint(fabsf(mu)));
+}
+
+// One CTA (128 threads) per (b, h, block); thread d owns channel d.
+// Residual codes E4M3((v - mean) * 448 / amax_d), stored transposed (each
+// thread writes its channel's 128 token codes, 128 contiguous bytes), and the
+// block's restore tile image.
+__global__ void __launch_bounds__(128)
+    v_quant_kernel(const __nv_bfloat16* __restrict__ v, Fp8Tensors t, int B, int H, int Skv) {
+    const int nkb = (Skv + kQuantBlock - 1) / kQuantBlock;
+    const int blk = blockIdx.x % nkb;
+    const int h = (blockIdx.x / nkb) % H;
+    const int b = blockIdx.x / (nkb * H);
+    const int d = threadIdx.x;
+    const int t0 = blk * kQuantBlock;
+    const int n = min(kQuantBlock, Skv - t0);
+    const size_t bh = static_cast<size_t>(b) * H + h;
+    const float amax = fmaxf(__uint_as_float(t.v_amax_r[bh * 128 + d]),
+                             __uint_as_float(t.v_amax_mu[bh * 128 + d]) * kMuFloor);
+    const float inv = amax > 0.0f ? kE4M3Max / amax : 0.0f;
+    if (blk == 0) t.v_scale[bh * 128 + d] = amax / kE4M3Max;
+    const float mu = t.mu[(bh * nkb + blk) * 128 + d];
+
+    const __nv_bfloat16* col = v + ((static_cast<size_t>(b) * Skv + t0) * H + h) * 128 + d;
+    const size_t stride = static_cast<size_t>(H) * 128;
+    uint4* out = reinterpret_cast<uint4*>(t.vt8 + ((bh * nkb + blk) * 128 + d) * 128);
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {  // 16 tokens per 16-byte store
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float r[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = g * 16 + e * 4 + u;
+                r[u] = i < n ? (__bfloat162float(col[i * stride]) - mu) * inv : 0.0f;
+            }
+            w[e] = e4m3x2(r[0], r[1]) | (e4m3x2(r[2], r[3]) << 16);
+        }
+        out[g] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+
+    // Restore tile: element (row k, channel d) of half d / 64 at
+    // k * 128 + ((c / 8) ^ (k & 7)) * 16 + (c % 8) * 2, c = d % 64.
+    __shared__ __align__(16) uint8_t img[kMuImgBytes];
+    for (int i = threadIdx.x; i < kMuImgBytes / 16; i += 128) reinterpret_cast<uint4*>(img)[i] = make_uint4(0, 0, 0, 0);
+    __syncthreads();
+    const float mu_p = mu * inv;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(mu_p);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(mu_p - __bfloat162float(hi));
+    const int half = d >> 6, c = d & 63;
+    const __nv_bfloat16 rows[3] = {hi, hi, lo};
+#pragma unroll
+    for (int kr = 0; kr < 3; ++kr)
+        *reinterpret_cast<__nv_bfloat16*>(img + half * 2048 + kr * 128 + (((c >> 3) ^ kr) << 4) + (c & 7) * 2) =
+            rows[kr];
+    __syncthreads();
+    uint4* img_out = reinterpret_cast<uint4*>(t.mu_img + (bh * nkb + blk) * kMuImgBytes);
+    for (int i = threadIdx.x; i < kMuImgBytes / 16; i += 128) img_out[i] = reinterpret_cast<const uint4*>(img)[i];
+}
+
+}  // namespace vdit

@@ -17,6 +17,8 @@
 #include "attn_fwd_sm100.cuh"
 #include "attn_merge.cuh"
 #include "qk_norm.cuh"
+#include "fp8_quant.cuh"
+#include "attn_fwd_fp8_sm100.cuh"
 
 namespace {
 
@@ -74,7 +76,9 @@ void init_device(int dev, DeviceState* st) {
         return;
     }
     if (cudaFuncSetAttribute(vdit::attn_fwd_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             vdit::kSmemBytes) != cudaSuccess) {
+                             vdit::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(vdit::attn_fwd_fp8_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             vdit::kF8SmemBytes) != cudaSuccess) {
         st->status = VDIT_ERR_CUDA;
         return;
     }
@@ -271,6 +275,168 @@ size_t qknorm_workspace_bytes(int B, int H, int Sq, int Skv, int D) {
     return round_up(size_t(B) * size_t(Sq) * row, kWorkspaceAlign) + size_t(B) * size_t(Skv) * row;
 }
 
+// ------------------------------------------------------------ 8-bit path
+
+// Byte offsets of the 8-bit path's workspace parts (the order of
+// VDIT_FP8_PART_* in the header), each 256-byte aligned; [VDIT_FP8_NUM_PARTS]
+// is the total.
+void fp8_layout(int B, int H, int Sq, int Skv, size_t* off) {
+    const size_t bh = size_t(B) * size_t(H);
+    const size_t nqb = size_t((Sq + vdit::kQuantBlock - 1) / vdit::kQuantBlock);
+    const size_t nkb = size_t((Skv + vdit::kQuantBlock - 1) / vdit::kQuantBlock);
+    const size_t sizes[VDIT_FP8_NUM_PARTS] = {
+        size_t(B) * size_t(Sq) * size_t(H) * 128,  // q8
+        size_t(B) * size_t(Skv) * size_t(H) * 128, // k8
+        bh * nkb * 128 * 128,                      // vt8
+        bh * nkb * vdit::kMuImgBytes,              // mu_img
+        bh * nqb * 4,                              // q_scale
+        bh * nkb * 4,                              // k_scale
+        bh * 128 * 4,                              // v_scale
+        bh * 128 * 4 * 2,                          // v_amax_r, v_amax_mu (zeroed together)
+        bh * nkb * 128 * 4,                        // mu
+    };
+    size_t at = 0;
+    for (int i = 0; i < VDIT_FP8_NUM_PARTS; ++i) {
+        off[i] = at;
+        at = round_up(at + sizes[i], kWorkspaceAlign);
+    }
+    off[VDIT_FP8_NUM_PARTS] = at;
+}
+
+vdit::Fp8Tensors fp8_tensors(void* ws, const size_t* off, int B, int H) {
+    char* w = static_cast<char*>(ws);
+    vdit::Fp8Tensors t;
+    t.q8 = reinterpret_cast<uint8_t*>(w + off[VDIT_FP8_PART_Q]);
+    t.k8 = reinterpret_cast<uint8_t*>(w + off[VDIT_FP8_PART_K]);
+    t.vt8 = reinterpret_cast<uint8_t*>(w + off[VDIT_FP8_PART_VT]);
+    t.mu_img = reinterpret_cast<uint8_t*>(w + off[VDIT_FP8_PART_MU_IMG]);
+    t.q_scale = reinterpret_cast<float*>(w + off[VDIT_FP8_PART_Q_SCALE]);
+    t.k_scale = reinterpret_cast<float*>(w + off[VDIT_FP8_PART_K_SCALE]);
+    t.v_scale = reinterpret_cast<float*>(w + off[VDIT_FP8_PART_V_SCALE]);
+    t.v_amax_r = reinterpret_cast<uint32_t*>(w + off[VDIT_FP8_PART_V_AMAX]);
+    t.v_amax_mu = t.v_amax_r + size_t(B) * size_t(H) * 128;
+    t.mu = reinterpret_cast<float*>(w + off[VDIT_FP8_PART_MU]);
+    return t;
+}
+
+// Shape and workspace checks shared by the 8-bit entry points.
+vdit_status fp8_check(const Shape& s, bool check_scale, float scale, void* workspace, size_t workspace_bytes,
+                      size_t* off) {
+    if (s.mask_kind == VDIT_MASK_BLOCK_SPARSE) return VDIT_ERR_INVALID_ARG;
+    vdit_status st = check_shape(s, check_scale, scale);
+    if (st != VDIT_OK) return st;
+    fp8_layout(s.B, s.H, s.Sq, s.Skv, off);
+    if (s.B == 0 || s.H == 0 || s.Sq == 0) return VDIT_OK;
+    if (workspace == nullptr || workspace_bytes < off[VDIT_FP8_NUM_PARTS]) return VDIT_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kWorkspaceAlign - 1)) != 0) return VDIT_ERR_MISALIGNED;
+    return VDIT_OK;
+}
+
+vdit_status fp8_quantize_impl(const void* q, const void* k, const void* v, const Shape& s, void* workspace,
+                              const size_t* off, cudaStream_t stream) {
+    if (q == nullptr || k == nullptr || v == nullptr) return VDIT_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return VDIT_ERR_MISALIGNED;
+    const size_t row = size_t(s.H) * 256;
+    const size_t qb = size_t(s.B) * size_t(s.Sq) * row, kb = size_t(s.B) * size_t(s.Skv) * row;
+    const size_t wb = off[VDIT_FP8_NUM_PARTS];
+    if (overlaps(workspace, wb, q, qb) || overlaps(workspace, wb, k, kb) || overlaps(workspace, wb, v, kb))
+        return VDIT_ERR_INVALID_ARG;
+    int dev = 0;
+    vdit_status st = ensure_device(&dev);
+    if (st != VDIT_OK) return st;
+    const vdit::Fp8Tensors t = fp8_tensors(workspace, off, s.B, s.H);
+    const long long nqb = (s.Sq + vdit::kQuantBlock - 1) / vdit::kQuantBlock;
+    const long long nkb = (s.Skv + vdit::kQuantBlock - 1) / vdit::kQuantBlock;
+    const long long bh = (long long)s.B * s.H;
+    if (bh * (nqb + nkb) > 0x7fffffffLL) return VDIT_ERR_INVALID_ARG;
+    if (cudaMemsetAsync(t.v_amax_r, 0, size_t(bh) * 128 * 4 * 2, stream) != cudaSuccess) return VDIT_ERR_CUDA;
+    vdit::qk_quant_kernel<<<unsigned(bh * (nqb + nkb)), 128, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), t, s.B, s.H, s.Sq, s.Skv);
+    vdit::v_stats_kernel<<<unsigned(bh * nkb), 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(v), t, s.B, s.H,
+                                                                 s.Skv);
+    vdit::v_quant_kernel<<<unsigned(bh * nkb), 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(v), t, s.B, s.H,
+                                                                 s.Skv);
+    return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
+}
+
+// E4M3 [B][S][H][128] codes as a 4-D tensor (128 bytes, H, S, B); a box is one
+// 128-token tile of one head, 128-byte swizzled.
+bool encode_bshd_u8(CUtensorMap* map, const void* base, int B, int S, int H) {
+    PFN_cuTensorMapEncodeTiled_v12000 f = encode_fn();
+    if (f == nullptr) return false;
+    cuuint64_t dims[4] = {128, cuuint64_t(H), cuuint64_t(S), cuuint64_t(B)};
+    cuuint64_t strides[3] = {128, cuuint64_t(H) * 128, cuuint64_t(S) * cuuint64_t(H) * 128};
+    cuuint32_t box[4] = {128, 1, cuuint32_t(vdit::kBlockM), 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return f(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The transposed V codes [blocks][128 channels][128 tokens] as a 3-D tensor.
+bool encode_vt_u8(CUtensorMap* map, const void* base, long long blocks) {
+    PFN_cuTensorMapEncodeTiled_v12000 f = encode_fn();
+    if (f == nullptr) return false;
+    cuuint64_t dims[3] = {128, 128, cuuint64_t(blocks)};
+    cuuint64_t strides[2] = {128, 128 * 128};
+    cuuint32_t box[3] = {128, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return f(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+vdit_status fp8_attention_impl(void* o, float* lse, const Shape& s, float scale, void* workspace,
+                               const size_t* off, cudaStream_t stream, bool after_quantize) {
+    if (o == nullptr) return VDIT_ERR_INVALID_ARG;
+    if (!aligned16(o) || !aligned16(lse)) return VDIT_ERR_MISALIGNED;
+    const size_t ob = size_t(s.B) * size_t(s.Sq) * size_t(s.H) * 256;
+    const size_t wb = off[VDIT_FP8_NUM_PARTS];
+    if (overlaps(o, ob, workspace, wb) ||
+        (lse != nullptr && (overlaps(lse, size_t(s.B) * s.H * s.Sq * 4, workspace, wb) ||
+                            overlaps(lse, size_t(s.B) * s.H * s.Sq * 4, o, ob))))
+        return VDIT_ERR_INVALID_ARG;
+    int dev = 0;
+    vdit_status st = ensure_device(&dev);
+    if (st != VDIT_OK) return st;
+    const vdit::Fp8Tensors t = fp8_tensors(workspace, off, s.B, s.H);
+    const int nqb = (s.Sq + vdit::kQuantBlock - 1) / vdit::kQuantBlock;
+    const int nkb = (s.Skv + vdit::kQuantBlock - 1) / vdit::kQuantBlock;
+    CUtensorMap tq, tk, tvt;
+    if (!encode_bshd_u8(&tq, t.q8, s.B, s.Sq, s.H) || !encode_bshd_u8(&tk, t.k8, s.B, s.Skv, s.H) ||
+        !encode_vt_u8(&tvt, t.vt8, (long long)s.B * s.H * nkb))
+        return VDIT_ERR_CUDA;
+    vdit::Fp8FwdParams p{};
+    p.B = s.B;
+    p.H = s.H;
+    p.Sq = s.Sq;
+    p.Skv = s.Skv;
+    p.mask_kind = s.mask_kind;
+    p.chunk = s.mask_kind == VDIT_MASK_BLOCK_CAUSAL ? s.chunk : 1;
+    p.c0 = static_cast<float>(8.0 * static_cast<double>(scale) * 1.4426950408889634);
+    p.q_scale = t.q_scale;
+    p.k_scale = t.k_scale;
+    p.v_scale = t.v_scale;
+    p.mu_img = t.mu_img;
+    p.nqb = nqb;
+    p.nkb = nkb;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.timeout_ns = kDefaultWaitTimeoutNs;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid_x(s.Sq), s.H, s.B);
+    cfg.blockDim = dim3(vdit::kNumThreads);
+    cfg.dynamicSmemBytes = vdit::kF8SmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = after_quantize ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, vdit::attn_fwd_fp8_sm100_kernel, tq, tk, tvt, p) == cudaSuccess ? VDIT_OK
+                                                                                                  : VDIT_ERR_CUDA;
+}
+
 }  // namespace
 
 // ------------------------------------------------------------ fixed scratch, no allocation
@@ -451,6 +617,83 @@ vdit_status vdit_attn_fwd_qknorm_noalloc(const void* q, const void* k, const voi
         // the normalised Q and K before the attention reads them.
         return vdit_attn_fwd_qknorm(q, k, v, o, lse, q_norm_weight, k_norm_weight, eps, B, H, Sq, Skv, D, scale,
                                     mask_kind, chunk_tokens, sc->ptr, size_t(VDIT_NOALLOC_SCRATCH_BYTES), stream);
+    } catch (...) {
+        return VDIT_ERR_CUDA;
+    }
+}
+
+vdit_status vdit_fp8_layout(int B, int H, int Sq, int Skv, int D, size_t* offsets) {
+    try {
+        if (offsets == nullptr) return VDIT_ERR_INVALID_ARG;
+        const Shape s{B, H, Sq, Skv, D, VDIT_MASK_FULL, 0};
+        const vdit_status st = check_shape(s, false, 1.0f);
+        if (st != VDIT_OK) return st;
+        fp8_layout(B, H, Sq, Skv, offsets);
+        return VDIT_OK;
+    } catch (...) {
+        return VDIT_ERR_INVALID_ARG;
+    }
+}
+
+vdit_status vdit_attn_fp8_plan(int B, int H, int Sq, int Skv, int D, int mask_kind, int chunk_tokens,
+                               size_t* workspace_bytes) {
+    try {
+        if (workspace_bytes == nullptr) return VDIT_ERR_INVALID_ARG;
+        size_t off[VDIT_FP8_NUM_PARTS + 1];
+        const Shape s{B, H, Sq, Skv, D, mask_kind, chunk_tokens};
+        const vdit_status st = fp8_check(s, false, 1.0f, nullptr, 0, off);
+        if (st != VDIT_OK && st != VDIT_ERR_WORKSPACE) return st;
+        *workspace_bytes = off[VDIT_FP8_NUM_PARTS];
+        return VDIT_OK;
+    } catch (...) {
+        return VDIT_ERR_INVALID_ARG;
+    }
+}
+
+vdit_status vdit_fp8_quantize(const void* q, const void* k, const void* v, int B, int H, int Sq, int Skv, int D,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    try {
+        size_t off[VDIT_FP8_NUM_PARTS + 1];
+        const Shape s{B, H, Sq, Skv, D, VDIT_MASK_FULL, 0};
+        const vdit_status st = fp8_check(s, false, 1.0f, workspace, workspace_bytes, off);
+        if (st != VDIT_OK || B == 0 || H == 0 || Sq == 0) return st;
+        return fp8_quantize_impl(q, k, v, s, workspace, off, static_cast<cudaStream_t>(stream));
+    } catch (...) {
+        return VDIT_ERR_CUDA;
+    }
+}
+
+vdit_status vdit_attn_fwd_fp8_quantized(void* o, float* lse, int B, int H, int Sq, int Skv, int D, float scale,
+                                        int mask_kind, int chunk_tokens, const void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+    try {
+        size_t off[VDIT_FP8_NUM_PARTS + 1];
+        const Shape s{B, H, Sq, Skv, D, mask_kind, chunk_tokens};
+        void* ws = const_cast<void*>(workspace);
+        const vdit_status st = fp8_check(s, true, scale, ws, workspace_bytes, off);
+        if (st != VDIT_OK || B == 0 || H == 0 || Sq == 0) return st;
+        return fp8_attention_impl(o, lse, s, scale, ws, off, static_cast<cudaStream_t>(stream), false);
+    } catch (...) {
+        return VDIT_ERR_CUDA;
+    }
+}
+
+vdit_status vdit_attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                              int Sq, int Skv, int D, float scale, int mask_kind, int chunk_tokens, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+    try {
+        size_t off[VDIT_FP8_NUM_PARTS + 1];
+        const Shape s{B, H, Sq, Skv, D, mask_kind, chunk_tokens};
+        vdit_status st = fp8_check(s, true, scale, workspace, workspace_bytes, off);
+        if (st != VDIT_OK || B == 0 || H == 0 || Sq == 0) return st;
+        if (o == nullptr) return VDIT_ERR_INVALID_ARG;
+        if (!aligned16(o) || !aligned16(lse)) return VDIT_ERR_MISALIGNED;
+        const size_t ob = size_t(B) * size_t(Sq) * size_t(H) * 256;
+        const size_t kb = size_t(B) * size_t(Skv) * size_t(H) * 256;
+        if (overlaps(o, ob, q, ob) || overlaps(o, ob, k, kb) || overlaps(o, ob, v, kb)) return VDIT_ERR_INVALID_ARG;
+        st = fp8_quantize_impl(q, k, v, s, workspace, off, static_cast<cudaStream_t>(stream));
+        if (st != VDIT_OK) return st;
+        return fp8_attention_impl(o, lse, s, scale, workspace, off, static_cast<cudaStream_t>(stream), true);
     } catch (...) {
         return VDIT_ERR_CUDA;
     }
