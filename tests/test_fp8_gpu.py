@@ -111,6 +111,22 @@ def test_fp8_attention_matches_its_oracle(B, H, Sq, Skv, mask, chunk, recipe):
     assert res["ok"], res
 
 
+def test_fp8_attention_with_a_wide_logit_span_takes_the_exact_clamp_and_matches():
+    # Q and K x30: |logit| reaches the thousands of code units, beyond what the
+    # 16-bit clamp may handle, so every warp runs the float-clamp loop
+    B, H, S = 1, 2, 600
+    q, k, v = wl.draw_qkv(B, H, S, S, 128, seed=96, recipe="iid")
+    q = (q.float() * 30).to(torch.bfloat16)
+    k = (k.float() * 30).to(torch.bfloat16)
+    scale = 1 / math.sqrt(128)
+    o, lse = _run_fp8(q, k, v, vb.VDIT_MASK_FULL, 0, scale)
+    o_r, l_r = f8.attention_fp8(wl.bf16_bits(q), wl.bf16_bits(k), wl.bf16_bits(v), scale)
+    og, lg = _flat(o, lse, B, H)
+    orr, lr = _flat(o_r, l_r, B, H)
+    res = check_parity(og, orr, lg, lr, [np.arange(i * S, (i + 1) * S) for i in range(B * H)], "fp8 wide span")
+    assert res["ok"], res
+
+
 def test_fp8_attention_is_close_to_exact_attention():
     B, H, S = 1, 2, 1000
     q, k, v = wl.draw_qkv(B, H, S, S, 128, seed=93, recipe="rms_qk_vout")

@@ -115,6 +115,13 @@ __device__ __forceinline__ void issue_pv_f8_half(uint32_t d_tmem, uint32_t p_tme
 
 // 32 scores -> 8 words of 4 ExpCast bytes, and the row-sum contribution in
 // 8 packed-fp16 accumulators (value * 2^-8 per byte).
+//
+// The FMA leaves t = 1.5 * 2^23 + y, so the low 16 bits of t are y whenever
+// -2^15 <= y < 2^15 (and 0 for t = -inf, a masked key).  kNarrow clamps y at 0
+// on those 16-bit lanes, two per instruction; that is exact when every score
+// of the row lies within 2^15 - 95 codes below the reference, which the caller
+// checks from the scales.  Otherwise t itself is clamped at 1.5 * 2^23 first.
+template <bool kNarrow>
 __device__ __forceinline__ void code_chunk(const uint32_t (&s)[32], uint64_t a2, uint64_t b2, uint32_t* pw,
                                            uint32_t (&acc)[8]) {
 #pragma unroll
@@ -122,15 +129,172 @@ __device__ __forceinline__ void code_chunk(const uint32_t (&s)[32], uint64_t a2,
         float t0, t1, t2, t3;
         ffma2(__uint_as_float(s[4 * q]), __uint_as_float(s[4 * q + 1]), a2, b2, t0, t1);
         ffma2(__uint_as_float(s[4 * q + 2]), __uint_as_float(s[4 * q + 3]), a2, b2, t2, t3);
-        t0 = fmaxf(t0, kMagic);
-        t1 = fmaxf(t1, kMagic);
-        t2 = fmaxf(t2, kMagic);
-        t3 = fmaxf(t3, kMagic);
-        const uint32_t h01 = prmt(__float_as_uint(t0), __float_as_uint(t1), 0x5410u);  // y0 | y1 << 16
-        const uint32_t h23 = prmt(__float_as_uint(t2), __float_as_uint(t3), 0x5410u);
-        pw[q] = prmt(h01, h23, 0x6420u);                                                 // y0 y1 y2 y3
+        uint32_t h01, h23;
+        if (kNarrow) {
+            h01 = max_s16x2(prmt(__float_as_uint(t0), __float_as_uint(t1), 0x5410u), 0u);
+            h23 = max_s16x2(prmt(__float_as_uint(t2), __float_as_uint(t3), 0x5410u), 0u);
+        } else {
+            h01 = prmt(__float_as_uint(fmaxf(t0, kMagic)), __float_as_uint(fmaxf(t1, kMagic)), 0x5410u);
+            h23 = prmt(__float_as_uint(fmaxf(t2, kMagic)), __float_as_uint(fmaxf(t3, kMagic)), 0x5410u);
+        }
+        pw[q] = prmt(h01, h23, 0x6420u);  // y0 y1 y2 y3  (h01 = y0 | y1 << 16)
         hadd2_acc(acc[q], h01 << 7);
         hadd2_acc(acc[q], h23 << 7);
+    }
+}
+
+// Largest |code product sum| of one score: 128 head dims x 448 x 448.
+constexpr float kF8MaxScoreCodes = 128.0f * 448.0f * 448.0f;
+
+// One query tile's softmax loop (the warp's 32 rows) over all key tiles, then
+// its epilogue.  Shared state lives in the kernel; see the kernel for roles.
+template <bool kNarrow>
+__device__ __forceinline__ void fp8_softmax_rows(const Fp8FwdParams& p, Fp8Barriers* bars, volatile int* abort_flag,
+                                                 int t, int lane, int row, size_t bh, uint32_t tS, uint32_t tO,
+                                                 int n_kv, int kv_lim, float cq) {
+    const uint32_t s_full = smem_addr(&bars->s_full[t]);
+    float ref_n = 0.0f;   // reference = ref_n + 0.65 (code units); set by the first tile
+    float l = 0.0f;       // running row sum in byte-value units at that reference
+    bool ok = true;
+    float sk_next = n_kv > 0 ? p.k_scale[bh * p.nkb] : 0.0f;
+    for (int j = 0; j < n_kv; ++j) {
+        const float sk = sk_next;
+        if (j + 1 < n_kv) sk_next = p.k_scale[bh * p.nkb + j + 1];  // hidden behind this tile
+        ok = warp_wait(s_full, uint32_t(j) & 1u, abort_flag, p.timeout_ns, kSiteSoftmax);
+        if (!ok) break;
+        tc_fence_after_sync();
+        uint32_t s[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + uint32_t(c) * 32u, s[c]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_wait(s[c]);
+        const int lim = kv_lim - j * kBlockN;
+        if (lim < kBlockN) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (c * 32 + i >= lim) s[c][i] = __float_as_uint(-INFINITY);
+        }
+        auto tile_max = [&]() {
+            float mxc[8];
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+                const uint32_t* v = &s[g >> 1][(g & 1) * 16];
+                float a = fmaxf(__uint_as_float(v[0]), __uint_as_float(v[1]));
+#pragma unroll
+                for (int i = 2; i < 16; i += 2) a = fmax3(a, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+                mxc[g] = a;
+            }
+            return fmax3(fmax3(mxc[0], mxc[1], mxc[2]), fmax3(mxc[3], mxc[4], mxc[5]), fmaxf(mxc[6], mxc[7]));
+        };
+        const float a = cq * sk;
+        const uint64_t a2 = pack_f32x2(a, a);
+        auto zmax_of = [&](float smax) { return smax == -INFINITY ? -INFINITY : smax * a; };
+        uint32_t acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        uint32_t pw[32];  // 128 bytes of P
+        if (j == 0) {
+            const float zmax = zmax_of(tile_max());
+            ref_n = zmax == -INFINITY ? 0.0f : ceilf(zmax - kF8RefFrac);
+            const float bc = kMagic + float(kF8CodeOffset) - ref_n;
+            const uint64_t b2 = pack_f32x2(bc, bc);
+            code_chunk<kNarrow>(s[0], a2, b2, pw, acc);
+            code_chunk<kNarrow>(s[1], a2, b2, pw + 8, acc);
+        } else {
+            {
+                const float bc = kMagic + float(kF8CodeOffset) - ref_n;
+                const uint64_t b2 = pack_f32x2(bc, bc);
+                code_chunk<kNarrow>(s[0], a2, b2, pw, acc);
+                code_chunk<kNarrow>(s[1], a2, b2, pw + 8, acc);
+            }
+            const float zmax = zmax_of(tile_max());
+            const bool rescale = zmax > ref_n + kF8RefFrac + kF8RescaleCodes;
+            if (__any_sync(0xffffffffu, rescale)) {
+                float alpha = 1.0f;
+                if (rescale) {
+                    const float new_n = ceilf(zmax - kF8RefFrac);
+                    alpha = ex2_approx((ref_n - new_n) * 0.125f);
+                    ref_n = new_n;
+                    l *= alpha;
+                    const float bc = kMagic + float(kF8CodeOffset) - ref_n;
+                    const uint64_t b2 = pack_f32x2(bc, bc);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) acc[q] = 0;
+                    code_chunk<kNarrow>(s[0], a2, b2, pw, acc);
+                    code_chunk<kNarrow>(s[1], a2, b2, pw + 8, acc);
+                }
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + uint32_t(c) * 32u, o);
+                    tmem_ld_wait(o);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st32(tO + uint32_t(c) * 32u, o);
+                }
+            }
+        }
+        // release keys 0-63
+        tmem_st16(tS, pw);
+        tmem_st_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(&bars->p_full[t][0]));
+        {
+            const float bc = kMagic + float(kF8CodeOffset) - ref_n;
+            const uint64_t b2 = pack_f32x2(bc, bc);
+            code_chunk<kNarrow>(s[2], a2, b2, pw + 16, acc);
+            code_chunk<kNarrow>(s[3], a2, b2, pw + 24, acc);
+        }
+        // l_j in byte-value units, and the restore operand [l_hi, l_lo, l_hi, 0 ...] (bf16)
+        float lj = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float2 f = f16x2_to_float2(acc[q]);
+            lj += f.x + f.y;
+        }
+        lj *= 256.0f;
+        l += lj;
+        const __nv_bfloat16 l_hi = __float2bfloat16_rn(lj);
+        const __nv_bfloat16 l_lo = __float2bfloat16_rn(lj - __bfloat162float(l_hi));
+        const uint32_t hi_bits = uint32_t(__bfloat16_as_ushort(l_hi));
+        uint32_t rop[8] = {hi_bits | (uint32_t(__bfloat16_as_ushort(l_lo)) << 16), hi_bits, 0, 0, 0, 0, 0, 0};
+        tmem_st16(tS + 16u, pw + 16);
+        tmem_st8(tS + 32u, rop);
+        tmem_st_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(&bars->p_full[t][1]));
+    }
+
+    if (ok && n_kv > 0) ok = warp_wait(smem_addr(&bars->o_full[t]), 0, abort_flag, p.timeout_ns, kSiteSoftmax);
+    if (ok) {
+        tc_fence_after_sync();
+        const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
+        const float* vs = p.v_scale + bh * kHeadDim;
+        const int b = int(bh / p.H), h = int(bh % p.H);
+        __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.Sq + row) * p.H + h) * kHeadDim;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + uint32_t(c) * 32u, o);
+            tmem_ld_wait(o);
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float2 sc = *reinterpret_cast<const float2*>(vs + c * 32 + 2 * i);
+                pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * (sc.x * inv_l),
+                                    __uint_as_float(o[2 * i + 1]) * (sc.y * inv_l));
+            }
+            if (row < p.Sq) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+        }
+        if (p.lse != nullptr && row < p.Sq)
+            p.lse[bh * p.Sq + row] = ((ref_n + kF8RefFrac) * 0.125f - kF8PShift + __log2f(l)) * 0.69314718055994531f;
     }
 }
 
@@ -296,7 +460,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const uint32_t lane_bits = uint32_t(quarter * 32) << 16;
         const uint32_t tS = tmem + lane_bits + uint32_t(t) * 128u;
         const uint32_t tO = tmem + lane_bits + 256u + uint32_t(t) * 128u;
-        const uint32_t s_full = smem_addr(&bars->s_full[t]);
 
         int kv_lim = p.Skv;
         if (p.mask_kind == kMaskBlockCausal) {
@@ -305,146 +468,19 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         }
         const int qblk = min(q0 / kBlockM + t, p.nqb - 1);
         const float cq = p.c0 * p.q_scale[bh * p.nqb + qblk];
-        float ref_n = 0.0f;   // reference = ref_n + 0.65 (code units); set by the first tile
-        float l = 0.0f;       // running row sum in byte-value units at that reference
-        bool ok = true;
-
-        for (int j = 0; j < n_kv; ++j) {
-            ok = warp_wait(s_full, uint32_t(j) & 1u, abort_flag, p.timeout_ns, kSiteSoftmax);
-            if (!ok) break;
-            tc_fence_after_sync();
-            uint32_t s[4][32];
+        // The 16-bit clamp is exact when no score of a row lies more than
+        // 2^15 - 95 codes below its reference; |score| <= cq * sk * 128 * 448^2,
+        // so a span bound of twice the largest such value (plus one code of
+        // reference rounding) below 32000 suffices.
+        float sk_max = 0.0f;
+        for (int i = lane; i < p.nkb; i += 32) sk_max = fmaxf(sk_max, p.k_scale[bh * p.nkb + i]);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tS + uint32_t(c) * 32u, s[c]);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld_wait(s[c]);
-            const int lim = kv_lim - j * kBlockN;
-            if (lim < kBlockN) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (c * 32 + i >= lim) s[c][i] = __float_as_uint(-INFINITY);
-            }
-            auto tile_max = [&]() {
-                float mxc[8];
-#pragma unroll
-                for (int g = 0; g < 8; ++g) {
-                    const uint32_t* v = &s[g >> 1][(g & 1) * 16];
-                    float a = fmaxf(__uint_as_float(v[0]), __uint_as_float(v[1]));
-#pragma unroll
-                    for (int i = 2; i < 16; i += 2) a = fmax3(a, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
-                    mxc[g] = a;
-                }
-                return fmax3(fmax3(mxc[0], mxc[1], mxc[2]), fmax3(mxc[3], mxc[4], mxc[5]), fmaxf(mxc[6], mxc[7]));
-            };
-            const float a = cq * p.k_scale[bh * p.nkb + j];
-            const uint64_t a2 = pack_f32x2(a, a);
-            auto zmax_of = [&](float smax) { return smax == -INFINITY ? -INFINITY : smax * a; };
-            uint32_t acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            uint32_t pw[32];  // 128 bytes of P
-            if (j == 0) {
-                const float zmax = zmax_of(tile_max());
-                ref_n = zmax == -INFINITY ? 0.0f : ceilf(zmax - kF8RefFrac);
-                const float bc = kMagic + float(kF8CodeOffset) - ref_n;
-                const uint64_t b2 = pack_f32x2(bc, bc);
-                code_chunk(s[0], a2, b2, pw, acc);
-                code_chunk(s[1], a2, b2, pw + 8, acc);
-            } else {
-                {
-                    const float bc = kMagic + float(kF8CodeOffset) - ref_n;
-                    const uint64_t b2 = pack_f32x2(bc, bc);
-                    code_chunk(s[0], a2, b2, pw, acc);
-                    code_chunk(s[1], a2, b2, pw + 8, acc);
-                }
-                const float zmax = zmax_of(tile_max());
-                const bool rescale = zmax > ref_n + kF8RefFrac + kF8RescaleCodes;
-                if (__any_sync(0xffffffffu, rescale)) {
-                    float alpha = 1.0f;
-                    if (rescale) {
-                        const float new_n = ceilf(zmax - kF8RefFrac);
-                        alpha = ex2_approx((ref_n - new_n) * 0.125f);
-                        ref_n = new_n;
-                        l *= alpha;
-                        const float bc = kMagic + float(kF8CodeOffset) - ref_n;
-                        const uint64_t b2 = pack_f32x2(bc, bc);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) acc[q] = 0;
-                        code_chunk(s[0], a2, b2, pw, acc);
-                        code_chunk(s[1], a2, b2, pw + 8, acc);
-                    }
-#pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + uint32_t(c) * 32u, o);
-                        tmem_ld_wait(o);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st32(tO + uint32_t(c) * 32u, o);
-                    }
-                }
-            }
-            // release keys 0-63
-            tmem_st16(tS, pw);
-            tmem_st_wait();
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&bars->p_full[t][0]));
-            {
-                const float bc = kMagic + float(kF8CodeOffset) - ref_n;
-                const uint64_t b2 = pack_f32x2(bc, bc);
-                code_chunk(s[2], a2, b2, pw + 16, acc);
-                code_chunk(s[3], a2, b2, pw + 24, acc);
-            }
-            // l_j in byte-value units, and the restore operand [l_hi, l_lo, l_hi, 0 ...] (bf16)
-            float lj = 0.0f;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float2 f = f16x2_to_float2(acc[q]);
-                lj += f.x + f.y;
-            }
-            lj *= 256.0f;
-            l += lj;
-            const __nv_bfloat16 l_hi = __float2bfloat16_rn(lj);
-            const __nv_bfloat16 l_lo = __float2bfloat16_rn(lj - __bfloat162float(l_hi));
-            const uint32_t hi_bits = uint32_t(__bfloat16_as_ushort(l_hi));
-            uint32_t rop[8] = {hi_bits | (uint32_t(__bfloat16_as_ushort(l_lo)) << 16), hi_bits, 0, 0, 0, 0, 0, 0};
-            tmem_st16(tS + 16u, pw + 16);
-            tmem_st8(tS + 32u, rop);
-            tmem_st_wait();
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&bars->p_full[t][1]));
-        }
-
-        if (ok && n_kv > 0) ok = warp_wait(smem_addr(&bars->o_full[t]), 0, abort_flag, p.timeout_ns, kSiteSoftmax);
-        if (ok) {
-            tc_fence_after_sync();
-            const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
-            const float* vs = p.v_scale + bh * kHeadDim;
-            __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.Sq + row) * p.H + h) * kHeadDim;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t o[32];
-                tmem_ld32(tO + uint32_t(c) * 32u, o);
-                tmem_ld_wait(o);
-                uint32_t pk[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float2 sc = *reinterpret_cast<const float2*>(vs + c * 32 + 2 * i);
-                    pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * (sc.x * inv_l),
-                                        __uint_as_float(o[2 * i + 1]) * (sc.y * inv_l));
-                }
-                if (row < p.Sq) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-                }
-            }
-            if (p.lse != nullptr && row < p.Sq)
-                p.lse[bh * p.Sq + row] = ((ref_n + kF8RefFrac) * 0.125f - kF8PShift + __log2f(l)) * 0.69314718055994531f;
-        }
+        for (int off = 16; off > 0; off >>= 1) sk_max = fmaxf(sk_max, __shfl_xor_sync(0xffffffffu, sk_max, off));
+        const bool narrow = 2.0f * cq * sk_max * kF8MaxScoreCodes + 2.0f < 32000.0f;
+        if (narrow)
+            fp8_softmax_rows<true>(p, bars, abort_flag, t, lane, row, bh, tS, tO, n_kv, kv_lim, cq);
+        else
+            fp8_softmax_rows<false>(p, bars, abort_flag, t, lane, row, bh, tS, tO, n_kv, kv_lim, cq);
     }
 
     tc_fence_before_sync();

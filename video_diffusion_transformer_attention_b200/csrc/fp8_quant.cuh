@@ -59,13 +59,17 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
     return uint32_t(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
 }
 
-// One CTA (128 threads) per (tensor, b, h, block).  Warp w holds tokens
-// 32w .. 32w+31 of the block; lane l holds channels 4l .. 4l+3 of each, so
+constexpr int kQuantThreads = 256;
+
+// One CTA (256 threads) per (tensor, b, h, block).  Warp w holds tokens
+// 16w .. 16w+15 of the block; lane l holds channels 4l .. 4l+3 of each, so
 // every load and store instruction of a warp covers one whole token row.
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kQuantThreads, 3)
     qk_quant_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, Fp8Tensors t,
                     int B, int H, int Sq, int Skv) {
-    __shared__ float warp_max[4];
+    constexpr int kWarps = kQuantThreads / 32;
+    constexpr int kTokPerWarp = kQuantBlock / kWarps;
+    __shared__ float warp_max[kWarps];
     const int nqb = (Sq + kQuantBlock - 1) / kQuantBlock;
     const int nkb = (Skv + kQuantBlock - 1) / kQuantBlock;
     long long id = blockIdx.x;
@@ -82,15 +86,19 @@ __global__ void __launch_bounds__(128)
     float* scale_out = is_k ? t.k_scale : t.q_scale;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tok0 = blk * kQuantBlock + warp * 32;
-    uint2 x[32];
+    const int tok0 = blk * kQuantBlock + warp * kTokPerWarp;
+    const size_t row_stride = static_cast<size_t>(H) * 128;  // elements between tokens
+    const size_t first = ((static_cast<size_t>(b) * S + tok0) * H + h) * 128 + lane * 4;
+    const int n_here = min(kTokPerWarp, S - tok0);
+    uint2 x[kTokPerWarp];
     float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const int tok = tok0 + i;
+    for (int i = 0; i < kTokPerWarp; ++i) {
         x[i] = make_uint2(0u, 0u);
-        if (tok < S)
-            x[i] = *reinterpret_cast<const uint2*>(src + ((static_cast<size_t>(b) * S + tok) * H + h) * 128 + lane * 4);
+        if (i < n_here) x[i] = __ldcs(reinterpret_cast<const uint2*>(src + first + i * row_stride));
+    }
+#pragma unroll
+    for (int i = 0; i < kTokPerWarp; ++i) {
         const __nv_bfloat162* v = reinterpret_cast<const __nv_bfloat162*>(&x[i]);
         const float2 f0 = __bfloat1622float2(v[0]), f1 = __bfloat1622float2(v[1]);
         amax = fmaxf(amax, fmaxf(fmaxf(fabsf(f0.x), fabsf(f0.y)), fmaxf(fabsf(f1.x), fabsf(f1.y))));
@@ -99,105 +107,128 @@ __global__ void __launch_bounds__(128)
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     if (lane == 0) warp_max[warp] = amax;
     __syncthreads();
-    amax = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) amax = fmaxf(amax, warp_max[w]);
     const float inv = amax > 0.0f ? kE4M3Max / amax : 0.0f;
     if (threadIdx.x == 0) scale_out[(static_cast<size_t>(b) * H + h) * nb + blk] = amax / kE4M3Max;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const int tok = tok0 + i;
-        if (tok >= S) break;
+    for (int i = 0; i < kTokPerWarp; ++i) {
+        if (i >= n_here) break;
         const __nv_bfloat162* v = reinterpret_cast<const __nv_bfloat162*>(&x[i]);
         const float2 f0 = __bfloat1622float2(v[0]), f1 = __bfloat1622float2(v[1]);
         const uint32_t c = e4m3x2(f0.x * inv, f0.y * inv) | (e4m3x2(f1.x * inv, f1.y * inv) << 16);
-        *reinterpret_cast<uint32_t*>(dst + ((static_cast<size_t>(b) * S + tok) * H + h) * 128 + lane * 4) = c;
+        *reinterpret_cast<uint32_t*>(dst + first + i * row_stride) = c;
     }
 }
 
-// One CTA (128 threads) per (b, h, block); thread d owns channel d.
-// Block mean (sequential fp32 sum over the block's tokens, then / n), the
-// block's largest |v - mean|, and the running per-channel maxima over the
-// head's blocks (atomicMax on the bits of non-negative floats, which order
-// like the floats).
-__global__ void __launch_bounds__(128)
+// Stage one (b, h) block of V ([128 tokens][128 channels] bf16, 32 KB) in
+// shared memory with whole-row loads (warp w loads tokens w, w+8, ...; lane l
+// loads channels 4l .. 4l+3); rows past Skv are zero.
+__device__ __forceinline__ void stage_v_block(const __nv_bfloat16* __restrict__ v, __nv_bfloat16* tile, int b, int h,
+                                              int H, int Skv, int t0, int n) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = warp; i < kQuantBlock; i += kQuantThreads / 32) {
+        uint2 x = make_uint2(0u, 0u);
+        if (i < n) x = __ldcs(reinterpret_cast<const uint2*>(v + ((static_cast<size_t>(b) * Skv + t0 + i) * H + h) * 128) + lane);
+        reinterpret_cast<uint2*>(tile + i * 128)[lane] = x;
+    }
+}
+
+// One CTA (256 threads) per (b, h, block); after staging, thread d < 128 owns
+// channel d: block mean (sequential fp32 sum over the block's tokens, then
+// / n), the block's largest |v - mean|, and the running per-channel maxima
+// over the head's blocks (atomicMax on the bits of non-negative floats,
+// which order like the floats).
+__global__ void __launch_bounds__(kQuantThreads)
     v_stats_kernel(const __nv_bfloat16* __restrict__ v, Fp8Tensors t, int B, int H, int Skv) {
+    __shared__ __align__(16) __nv_bfloat16 tile[kQuantBlock * 128];
     const int nkb = (Skv + kQuantBlock - 1) / kQuantBlock;
     const int blk = blockIdx.x % nkb;
     const int h = (blockIdx.x / nkb) % H;
     const int b = blockIdx.x / (nkb * H);
-    const int d = threadIdx.x;
     const int t0 = blk * kQuantBlock;
     const int n = min(kQuantBlock, Skv - t0);
-    const __nv_bfloat16* col = v + ((static_cast<size_t>(b) * Skv + t0) * H + h) * 128 + d;
-    const size_t stride = static_cast<size_t>(H) * 128;
+    stage_v_block(v, tile, b, h, H, Skv, t0, n);
+    __syncthreads();
+    const int d = threadIdx.x;
+    if (d >= 128) return;
     float sum = 0.0f;
-#pragma unroll 16
-    for (int i = 0; i < n; ++i) sum += __bfloat162float(col[i * stride]);
+    for (int i = 0; i < n; ++i) sum += __bfloat162float(tile[i * 128 + d]);
     const float mu = sum / static_cast<float>(n);
     float rmax = 0.0f;
-#pragma unroll 16
-    for (int i = 0; i < n; ++i) rmax = fmaxf(rmax, fabsf(__bfloat162float(col[i * stride]) - mu));
+    for (int i = 0; i < n; ++i) rmax = fmaxf(rmax, fabsf(__bfloat162float(tile[i * 128 + d]) - mu));
     const size_t bh = static_cast<size_t>(b) * H + h;
     t.mu[(bh * nkb + blk) * 128 + d] = mu;
     atomicMax(t.v_amax_r + bh * 128 + d, __float_as_uint(rmax));
     atomicMax(t.v_amax_mu + bh * 128 + d, __float_as_uint(fabsf(mu)));
 }
 
-// One CTA (128 threads) per (b, h, block); thread d owns channel d.
-// Residual codes E4M3((v - mean) * 448 / amax_d), stored transposed (each
-// thread writes its channel's 128 token codes, 128 contiguous bytes), and the
-// block's restore tile image.
-__global__ void __launch_bounds__(128)
+// One CTA (256 threads) per (b, h, block).  After staging, thread d < 128
+// computes the residual codes E4M3((v - mean) * 448 / amax_d) of channel d
+// into a transposed shared-memory tile ([channel][token] bytes), which the
+// whole CTA then writes out as contiguous 16-byte rows; threads 128-255 write
+// the block's restore tile meanwhile (rows 3-15 zero as 16-byte stores, rows
+// 0-2 one bf16 per thread).
+__global__ void __launch_bounds__(kQuantThreads)
     v_quant_kernel(const __nv_bfloat16* __restrict__ v, Fp8Tensors t, int B, int H, int Skv) {
+    __shared__ __align__(16) __nv_bfloat16 tile[kQuantBlock * 128];
+    __shared__ __align__(16) uint8_t codes[128 * kQuantBlock];
     const int nkb = (Skv + kQuantBlock - 1) / kQuantBlock;
     const int blk = blockIdx.x % nkb;
     const int h = (blockIdx.x / nkb) % H;
     const int b = blockIdx.x / (nkb * H);
-    const int d = threadIdx.x;
     const int t0 = blk * kQuantBlock;
     const int n = min(kQuantBlock, Skv - t0);
     const size_t bh = static_cast<size_t>(b) * H + h;
+    stage_v_block(v, tile, b, h, H, Skv, t0, n);
+    __syncthreads();
+    uint8_t* img = t.mu_img + (bh * nkb + blk) * kMuImgBytes;
+    const int d = threadIdx.x & 127;
     const float amax = fmaxf(__uint_as_float(t.v_amax_r[bh * 128 + d]),
                              __uint_as_float(t.v_amax_mu[bh * 128 + d]) * kMuFloor);
     const float inv = amax > 0.0f ? kE4M3Max / amax : 0.0f;
-    if (blk == 0) t.v_scale[bh * 128 + d] = amax / kE4M3Max;
     const float mu = t.mu[(bh * nkb + blk) * 128 + d];
-
-    const __nv_bfloat16* col = v + ((static_cast<size_t>(b) * Skv + t0) * H + h) * 128 + d;
-    const size_t stride = static_cast<size_t>(H) * 128;
-    uint4* out = reinterpret_cast<uint4*>(t.vt8 + ((bh * nkb + blk) * 128 + d) * 128);
+    if (threadIdx.x < 128) {
+        if (blk == 0) t.v_scale[bh * 128 + d] = amax / kE4M3Max;
+        // 16 tokens per 16-byte word; the word index is rotated by the channel so
+        // that the 32 lanes of a warp store to different banks
+#pragma unroll 1
+        for (int gi = 0; gi < 8; ++gi) {
+            const int g = (gi + (d >> 2)) & 7;
+            uint32_t w[4];
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {  // 16 tokens per 16-byte store
-        uint32_t w[4];
+            for (int e = 0; e < 4; ++e) {
+                float r[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            float r[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int i = g * 16 + e * 4 + u;
-                r[u] = i < n ? (__bfloat162float(col[i * stride]) - mu) * inv : 0.0f;
+                for (int u = 0; u < 4; ++u) {
+                    const int i = g * 16 + e * 4 + u;
+                    r[u] = i < n ? (__bfloat162float(tile[i * 128 + d]) - mu) * inv : 0.0f;
+                }
+                w[e] = e4m3x2(r[0], r[1]) | (e4m3x2(r[2], r[3]) << 16);
             }
-            w[e] = e4m3x2(r[0], r[1]) | (e4m3x2(r[2], r[3]) << 16);
+            reinterpret_cast<uint4*>(codes + d * kQuantBlock)[g] = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        out[g] = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-
-    // Restore tile: element (row k, channel d) of half d / 64 at
-    // k * 128 + ((c / 8) ^ (k & 7)) * 16 + (c % 8) * 2, c = d % 64.
-    __shared__ __align__(16) uint8_t img[kMuImgBytes];
-    for (int i = threadIdx.x; i < kMuImgBytes / 16; i += 128) reinterpret_cast<uint4*>(img)[i] = make_uint4(0, 0, 0, 0);
-    __syncthreads();
-    const float mu_p = mu * inv;
-    const __nv_bfloat16 hi = __float2bfloat16_rn(mu_p);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(mu_p - __bfloat162float(hi));
-    const int half = d >> 6, c = d & 63;
-    const __nv_bfloat16 rows[3] = {hi, hi, lo};
+    } else {
+        // zero rows 3-15 of both halves: 2 x 13 rows x 8 chunks of 16 bytes
+        for (int i = threadIdx.x - 128; i < 2 * 13 * 8; i += 128) {
+            const int half = i / (13 * 8), r = 3 + (i / 8) % 13, ch = i % 8;
+            *reinterpret_cast<uint4*>(img + half * 2048 + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+        }
+        // Restore tile: element (row k, channel d) of half d / 64 at
+        // k * 128 + ((c / 8) ^ (k & 7)) * 16 + (c % 8) * 2, c = d % 64.
+        const float mu_p = mu * inv;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(mu_p);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(mu_p - __bfloat162float(hi));
+        const int half = d >> 6, c = d & 63;
+        const __nv_bfloat16 rows[3] = {hi, hi, lo};
 #pragma unroll
-    for (int kr = 0; kr < 3; ++kr)
-        *reinterpret_cast<__nv_bfloat16*>(img + half * 2048 + kr * 128 + (((c >> 3) ^ kr) << 4) + (c & 7) * 2) =
-            rows[kr];
+        for (int kr = 0; kr < 3; ++kr)
+            *reinterpret_cast<__nv_bfloat16*>(img + half * 2048 + kr * 128 + (((c >> 3) ^ kr) << 4) + (c & 7) * 2) =
+                rows[kr];
+    }
     __syncthreads();
-    uint4* img_out = reinterpret_cast<uint4*>(t.mu_img + (bh * nkb + blk) * kMuImgBytes);
-    for (int i = threadIdx.x; i < kMuImgBytes / 16; i += 128) img_out[i] = reinterpret_cast<const uint4*>(img)[i];
+    uint4* out = reinterpret_cast<uint4*>(t.vt8 + (bh * nkb + blk) * 128 * kQuantBlock);
+    for (int i = threadIdx.x; i < 128 * kQuantBlock / 16; i += kQuantThreads) out[i] = reinterpret_cast<const uint4*>(codes)[i];
 }
 
 }  // namespace vdit

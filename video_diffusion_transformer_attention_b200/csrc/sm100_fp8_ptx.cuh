@@ -62,6 +62,13 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return d;
 }
 
+// Lane-wise maximum of two pairs of signed 16-bit integers.
+__device__ __forceinline__ uint32_t max_s16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.s16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
 // acc += x, two packed fp16 lanes.
 __device__ __forceinline__ void hadd2_acc(uint32_t& acc, uint32_t x) {
     asm("add.rn.f16x2 %0, %0, %1;" : "+r"(acc) : "r"(x));

@@ -350,11 +350,11 @@ vdit_status fp8_quantize_impl(const void* q, const void* k, const void* v, const
     const long long bh = (long long)s.B * s.H;
     if (bh * (nqb + nkb) > 0x7fffffffLL) return VDIT_ERR_INVALID_ARG;
     if (cudaMemsetAsync(t.v_amax_r, 0, size_t(bh) * 128 * 4 * 2, stream) != cudaSuccess) return VDIT_ERR_CUDA;
-    vdit::qk_quant_kernel<<<unsigned(bh * (nqb + nkb)), 128, 0, stream>>>(
+    vdit::qk_quant_kernel<<<unsigned(bh * (nqb + nkb)), vdit::kQuantThreads, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), t, s.B, s.H, s.Sq, s.Skv);
-    vdit::v_stats_kernel<<<unsigned(bh * nkb), 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(v), t, s.B, s.H,
+    vdit::v_stats_kernel<<<unsigned(bh * nkb), vdit::kQuantThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(v), t, s.B, s.H,
                                                                  s.Skv);
-    vdit::v_quant_kernel<<<unsigned(bh * nkb), 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(v), t, s.B, s.H,
+    vdit::v_quant_kernel<<<unsigned(bh * nkb), vdit::kQuantThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(v), t, s.B, s.H,
                                                                  s.Skv);
     return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
 }
