@@ -289,6 +289,43 @@ vdit_status vdit_attn_fwd_fp8(const void* q, const void* k, const void* v,
                               size_t workspace_bytes, void* stream);
 
 /*
+ * V-Smooth "Group" (VC-Attention (aikraft.ru), section 02): cluster the value
+ * tokens of every (batch, head) with a k-means warm-started from the caller's
+ * centroids (the previous denoising step's), then permute K and V together
+ * so that each cluster's tokens are adjacent.  A joint K/V permutation leaves
+ * non-causal attention (FULL, CROSS) unchanged, and the 128-token blocks of
+ * the permuted sequence have block means that remove more of V before the
+ * 8-bit path quantises it.  Not for BLOCK_CAUSAL.
+ *
+ * vdit_vsmooth_group runs `iters` Lloyd iterations (assign each token to its
+ * nearest centroid in squared Euclidean distance, lowest index on ties; move
+ * each centroid to the mean of its tokens, keeping centroids without tokens),
+ * then assigns once more and sorts stably by cluster:
+ *   v          device bf16 [B][S][H][128]
+ *   centroids  device fp32 [B][H][C][128], read and updated in place
+ *   labels     device int32 [B][H][S], the final assignment
+ *   perm       device int32 [B][H][S]: perm[b][h][i] = the token at position i
+ *   C          1 .. 64 clusters
+ *   workspace  device, vdit_vsmooth_group_plan bytes, 256-byte aligned (may be
+ *              NULL when iters == 0)
+ * Centroid sums use float atomics, so centroids may differ in the last bits
+ * from run to run; labels and perm are then the exact consequence of them.
+ */
+vdit_status vdit_vsmooth_group_plan(int B, int H, int S, int D, int C,
+                                    size_t* workspace_bytes);
+vdit_status vdit_vsmooth_group(const void* v, float* centroids,
+                               int32_t* labels, int32_t* perm, int B, int H,
+                               int S, int D, int C, int iters,
+                               void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* k_out[b][i][h][:] = k[b][perm[b][h][i]][h][:], the same for v (bf16,
+ * [B][S][H][128]).  Outputs must not overlap any input. */
+vdit_status vdit_permute_kv(const void* k, const void* v, const int32_t* perm,
+                            void* k_out, void* v_out, int B, int H, int S,
+                            int D, void* stream);
+
+/*
  * vdit_attn_fwd_ws -- vdit_attn_fwd with a caller-owned device workspace of
  * `workspace_bytes` bytes (at least what vdit_attn_plan reports; NULL is
  * accepted when that is 0).

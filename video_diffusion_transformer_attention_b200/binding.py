@@ -48,6 +48,9 @@ EXPORTS = (
     "vdit_fp8_quantize",
     "vdit_attn_fwd_fp8_quantized",
     "vdit_attn_fwd_fp8",
+    "vdit_vsmooth_group_plan",
+    "vdit_vsmooth_group",
+    "vdit_permute_kv",
     "vdit_get_device_status",
     "vdit_status_string",
     "vdit_abi_version",
@@ -105,6 +108,12 @@ def lib() -> ctypes.CDLL:
             h.vdit_attn_fwd_fp8_quantized.argtypes = [vp, vp] + [c_int] * 5 + [c_float, c_int, c_int, vp, c_size, vp]
             h.vdit_attn_fwd_fp8.restype = c_int
             h.vdit_attn_fwd_fp8.argtypes = fwd_args + [vp, c_size, vp]
+            h.vdit_vsmooth_group_plan.restype = c_int
+            h.vdit_vsmooth_group_plan.argtypes = [c_int] * 5 + [ctypes.POINTER(c_size)]
+            h.vdit_vsmooth_group.restype = c_int
+            h.vdit_vsmooth_group.argtypes = [vp, vp, vp, vp] + [c_int] * 6 + [vp, c_size, vp]
+            h.vdit_permute_kv.restype = c_int
+            h.vdit_permute_kv.argtypes = [vp] * 5 + [c_int] * 4 + [vp]
             h.vdit_qk_rms_norm.restype = c_int
             h.vdit_qk_rms_norm.argtypes = [vp, vp, vp, vp, vp, vp, c_float, c_int, c_int, c_int, c_int, c_int, vp]
             h.vdit_attn_merge.restype = c_int
@@ -280,6 +289,54 @@ def attention_fp8(q, k, v, scale=None, mask_kind=VDIT_MASK_FULL, chunk_tokens=0,
     vdit_attn_fwd_fp8(q, k, v, out, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, workspace,
                       workspace.numel(), stream)
     return out, lse, workspace
+
+
+def vdit_vsmooth_group_plan(B, H, S, D, C):
+    ws = ctypes.c_size_t(0)
+    st = lib().vdit_vsmooth_group_plan(B, H, S, D, C, ctypes.byref(ws))
+    return int(st), int(ws.value)
+
+
+def vdit_vsmooth_group(v, centroids, labels, perm, B, H, S, D, C, iters, workspace, workspace_bytes, stream=None,
+                       check=True) -> int:
+    st = lib().vdit_vsmooth_group(_addr(v), _addr(centroids), _addr(labels), _addr(perm), B, H, S, D, C, iters,
+                                  _addr(workspace), int(workspace_bytes), _stream(stream))
+    if check and st != VDIT_OK:
+        raise VditError(st, "vdit_vsmooth_group")
+    return st
+
+
+def vdit_permute_kv(k, v, perm, k_out, v_out, B, H, S, D, stream=None, check=True) -> int:
+    st = lib().vdit_permute_kv(_addr(k), _addr(v), _addr(perm), _addr(k_out), _addr(v_out), B, H, S, D,
+                               _stream(stream))
+    if check and st != VDIT_OK:
+        raise VditError(st, "vdit_permute_kv")
+    return st
+
+
+def vsmooth_group(v, centroids, iters=4, stream=None):
+    """Group step on CUDA tensors: v bf16 [B, S, H, 128], centroids fp32 [B, H, C, 128] (updated in place).
+    Returns (labels, perm), int32 [B, H, S]."""
+    import torch
+    B, S, H, D = v.shape
+    C = centroids.shape[2]
+    st, need = vdit_vsmooth_group_plan(B, H, S, D, C)
+    if st != VDIT_OK:
+        raise VditError(st, "vdit_vsmooth_group_plan")
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=v.device)
+    labels = torch.empty((B, H, S), dtype=torch.int32, device=v.device)
+    perm = torch.empty((B, H, S), dtype=torch.int32, device=v.device)
+    vdit_vsmooth_group(v, centroids, labels, perm, B, H, S, D, C, iters, ws, ws.numel(), stream)
+    return labels, perm
+
+
+def permute_kv(k, v, perm, stream=None):
+    """K and V gathered per head by perm (CUDA bf16 [B, S, H, 128], perm int32 [B, H, S])."""
+    import torch
+    B, S, H, D = k.shape
+    k_out, v_out = torch.empty_like(k), torch.empty_like(v)
+    vdit_permute_kv(k, v, perm, k_out, v_out, B, H, S, D, stream)
+    return k_out, v_out
 
 
 NOALLOC_SCRATCH_BYTES = 64 << 20  # VDIT_NOALLOC_SCRATCH_BYTES in include/vdit_attn.h

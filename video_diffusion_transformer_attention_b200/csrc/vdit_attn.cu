@@ -19,6 +19,7 @@
 #include "qk_norm.cuh"
 #include "fp8_quant.cuh"
 #include "attn_fwd_fp8_sm100.cuh"
+#include "vsmooth_group.cuh"
 
 namespace {
 
@@ -694,6 +695,100 @@ vdit_status vdit_attn_fwd_fp8(const void* q, const void* k, const void* v, void*
         st = fp8_quantize_impl(q, k, v, s, workspace, off, static_cast<cudaStream_t>(stream));
         if (st != VDIT_OK) return st;
         return fp8_attention_impl(o, lse, s, scale, workspace, off, static_cast<cudaStream_t>(stream), true);
+    } catch (...) {
+        return VDIT_ERR_CUDA;
+    }
+}
+
+vdit_status vdit_vsmooth_group_plan(int B, int H, int S, int D, int C, size_t* workspace_bytes) {
+    try {
+        if (workspace_bytes == nullptr || B < 0 || H < 0 || S < 0 || D < 1) return VDIT_ERR_INVALID_ARG;
+        if (D != 128) return VDIT_ERR_UNSUPPORTED;
+        if (C < 1 || C > vdit::kGroupMaxClusters) return VDIT_ERR_INVALID_ARG;
+        const size_t bhc = size_t(B) * size_t(H) * size_t(C);
+        *workspace_bytes = round_up(bhc * 128 * 4, kWorkspaceAlign) + bhc * 4;
+        return VDIT_OK;
+    } catch (...) {
+        return VDIT_ERR_INVALID_ARG;
+    }
+}
+
+vdit_status vdit_vsmooth_group(const void* v, float* centroids, int32_t* labels, int32_t* perm, int B, int H, int S,
+                               int D, int C, int iters, void* workspace, size_t workspace_bytes, void* stream) {
+    try {
+        size_t need = 0;
+        vdit_status st = vdit_vsmooth_group_plan(B, H, S, D, C, &need);
+        if (st != VDIT_OK) return st;
+        if (iters < 0 || iters > 1000) return VDIT_ERR_INVALID_ARG;
+        if (B > 65535 || H > 65535) return VDIT_ERR_INVALID_ARG;
+        if (B == 0 || H == 0 || S == 0) return VDIT_OK;
+        if (v == nullptr || centroids == nullptr || labels == nullptr || perm == nullptr)
+            return VDIT_ERR_INVALID_ARG;
+        if (!aligned16(v) || !aligned16(centroids) || (reinterpret_cast<uintptr_t>(labels) & 3) ||
+            (reinterpret_cast<uintptr_t>(perm) & 3))
+            return VDIT_ERR_MISALIGNED;
+        if (iters > 0) {
+            if (workspace == nullptr || workspace_bytes < need) return VDIT_ERR_WORKSPACE;
+            if ((reinterpret_cast<uintptr_t>(workspace) & (kWorkspaceAlign - 1)) != 0) return VDIT_ERR_MISALIGNED;
+        }
+        const size_t bh = size_t(B) * size_t(H);
+        const size_t vb = bh * size_t(S) * 256, cb = bh * size_t(C) * 512, lb = bh * size_t(S) * 4;
+        if (overlaps(centroids, cb, v, vb) || overlaps(labels, lb, v, vb) || overlaps(perm, lb, v, vb) ||
+            overlaps(labels, lb, perm, lb) || overlaps(labels, lb, centroids, cb) ||
+            overlaps(perm, lb, centroids, cb) ||
+            (iters > 0 && (overlaps(workspace, need, v, vb) || overlaps(workspace, need, centroids, cb) ||
+                           overlaps(workspace, need, labels, lb) || overlaps(workspace, need, perm, lb))))
+            return VDIT_ERR_INVALID_ARG;
+        int dev = 0;
+        st = ensure_device(&dev);
+        if (st != VDIT_OK) return st;
+        cudaStream_t sm = static_cast<cudaStream_t>(stream);
+        const __nv_bfloat16* vv = static_cast<const __nv_bfloat16*>(v);
+        float* sums = static_cast<float*>(workspace);
+        int32_t* counts = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) +
+                                                     round_up(bh * size_t(C) * 512, kWorkspaceAlign));
+        const dim3 grid((S + vdit::kGroupTokens - 1) / vdit::kGroupTokens, H, B);
+        for (int it = 0; it < iters; ++it) {
+            vdit::group_assign_kernel<<<grid, vdit::kGroupTokens, 0, sm>>>(vv, centroids, labels, H, S, C);
+            if (cudaMemsetAsync(workspace, 0, need, sm) != cudaSuccess) return VDIT_ERR_CUDA;
+            vdit::group_accumulate_kernel<<<grid, 128, 0, sm>>>(vv, labels, sums, counts, H, S, C);
+            vdit::group_finalize_kernel<<<unsigned(bh * size_t(C)), 128, 0, sm>>>(sums, counts, centroids, C);
+        }
+        vdit::group_assign_kernel<<<grid, vdit::kGroupTokens, 0, sm>>>(vv, centroids, labels, H, S, C);
+        vdit::group_sort_kernel<<<unsigned(bh), vdit::kSortThreads, 0, sm>>>(labels, perm, S, C);
+        return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
+    } catch (...) {
+        return VDIT_ERR_CUDA;
+    }
+}
+
+vdit_status vdit_permute_kv(const void* k, const void* v, const int32_t* perm, void* k_out, void* v_out, int B,
+                            int H, int S, int D, void* stream) {
+    try {
+        if (B < 0 || H < 0 || S < 0 || D < 1) return VDIT_ERR_INVALID_ARG;
+        if (D != 128) return VDIT_ERR_UNSUPPORTED;
+        if (B == 0 || H == 0 || S == 0) return VDIT_OK;
+        if (k == nullptr || v == nullptr || perm == nullptr || k_out == nullptr || v_out == nullptr)
+            return VDIT_ERR_INVALID_ARG;
+        if (!aligned16(k) || !aligned16(v) || !aligned16(k_out) || !aligned16(v_out) ||
+            (reinterpret_cast<uintptr_t>(perm) & 3))
+            return VDIT_ERR_MISALIGNED;
+        const size_t tb = size_t(B) * size_t(S) * size_t(H) * 256, pb = size_t(B) * size_t(H) * size_t(S) * 4;
+        const void* ins[3] = {k, v, perm};
+        const size_t in_b[3] = {tb, tb, pb};
+        for (int i = 0; i < 3; ++i)
+            if (overlaps(k_out, tb, ins[i], in_b[i]) || overlaps(v_out, tb, ins[i], in_b[i])) return VDIT_ERR_INVALID_ARG;
+        if (overlaps(k_out, tb, v_out, tb)) return VDIT_ERR_INVALID_ARG;
+        int dev = 0;
+        const vdit_status st = ensure_device(&dev);
+        if (st != VDIT_OK) return st;
+        const long long rows = (long long)B * H * S;
+        const long long blocks = (rows * 16 + 255) / 256;
+        if (blocks > 0x7fffffffLL) return VDIT_ERR_INVALID_ARG;
+        vdit::permute_rows_kernel<<<unsigned(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+            static_cast<const uint4*>(k), static_cast<const uint4*>(v), perm, static_cast<uint4*>(k_out),
+            static_cast<uint4*>(v_out), H, S, rows);
+        return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
     } catch (...) {
         return VDIT_ERR_CUDA;
     }
