@@ -301,12 +301,14 @@ def run_vdit(args):
             vb.vdit_attn_fwd(q, k, v, o, lse, call.B, call.H, call.Sq, call.Skv, call.D, call.scale,
                              call.mask_kind, call.chunk_tokens, sptr)
 
-    def step(events=None):
+    def step(events=None, inp_set=None, out_set=None):
+        inp_set = inp if inp_set is None else inp_set
+        out_set = outs if out_set is None else out_set
         for i, call in enumerate(w.calls):
-            q, k, v = call_inputs(inp, call)
+            q, k, v = call_inputs(inp_set, call)
             if events is not None:
                 events[i][0].record(stream)
-            launch(i, call, q, k, v, *outs[i], mid_event=events[i][2] if events is not None else None)
+            launch(i, call, q, k, v, *out_set[i], mid_event=events[i][2] if events is not None else None)
             if events is not None:
                 events[i][1].record(stream)
 
@@ -350,6 +352,10 @@ def run_vdit(args):
     value = job_tflops(world, step_flops, args.steps, ms_max)
 
     # ---- end to end through the public API, host buffers in and out
+    # Every step copies its inputs from pinned host memory and its results back.
+    # Three streams pipeline consecutive steps over two device buffer sets:
+    # while step i computes, step i+1's inputs go up and step i-1's results
+    # come down (separate copy engines, each direction at full PCIe rate).
     e2e = None
     if args.e2e_steps > 0:
         host_in = {k: v.pin_memory() for k, v in inp_cpu.items()}
@@ -357,30 +363,54 @@ def run_vdit(args):
                     for o, l in outs]
         h2d = sum(t.numel() * t.element_size() for t in host_in.values())
         d2h = sum(o.numel() * o.element_size() + l.numel() * l.element_size() for o, l in host_out)
+        inp_sets = [inp, {k: torch.empty_like(v) for k, v in inp.items()}]
+        out_sets = [outs, [(torch.empty_like(o), torch.empty_like(l)) for o, l in outs]]
+        s_in = torch.cuda.Stream(device=dev)
+        s_out = torch.cuda.Stream(device=dev)
+        ev = {name: [torch.cuda.Event() for _ in range(2)] for name in ("in_ready", "in_free", "out_ready", "out_free")}
 
-        def e2e_step():
-            with torch.cuda.stream(stream):
-                for k_, v_ in host_in.items():
-                    inp[k_].copy_(v_, non_blocking=True)
-                step()
-                for (o, l), (ho, hl) in zip(outs, host_out):
-                    ho.copy_(o, non_blocking=True)
-                    hl.copy_(l, non_blocking=True)
+        def pipelined(n_steps):
+            for i in range(n_steps):
+                b = i % 2
+                if i >= 2:
+                    s_in.wait_event(ev["in_free"][b])
+                with torch.cuda.stream(s_in):
+                    for k_, v_ in host_in.items():
+                        inp_sets[b][k_].copy_(v_, non_blocking=True)
+                ev["in_ready"][b].record(s_in)
+                stream.wait_event(ev["in_ready"][b])
+                if i >= 2:
+                    stream.wait_event(ev["out_free"][b])
+                with torch.cuda.stream(stream):
+                    step(inp_set=inp_sets[b], out_set=out_sets[b])
+                ev["in_free"][b].record(stream)
+                ev["out_ready"][b].record(stream)
+                s_out.wait_event(ev["out_ready"][b])
+                with torch.cuda.stream(s_out):
+                    for (o, l), (ho, hl) in zip(out_sets[b], host_out):
+                        ho.copy_(o, non_blocking=True)
+                        hl.copy_(l, non_blocking=True)
+                ev["out_free"][b].record(s_out)
 
-        e2e_step()
-        stream.synchronize()
+        pipelined(2)
+        torch.cuda.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        e1.record(stream)
-        stream.synchronize()
+        e0.record(s_in)
+        stream.wait_event(e0)
+        s_out.wait_event(e0)
+        pipelined(args.e2e_steps)
+        e1.record(s_out)
+        torch.cuda.synchronize()
         barrier()
         e_ms = reduce_max(e0.elapsed_time(e1), dist, dev)
         e2e = {"value": job_tflops(world, step_flops, args.e2e_steps, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps}
+               "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps,
+               "overlap": "inputs of step i+1 up and results of step i-1 down while step i computes"}
+        st, word = vb.vdit_get_device_status(sptr)
+        if st != vb.VDIT_OK:
+            raise SystemExit(f"device status after the end-to-end steps: {vb.vdit_status_string(st)} ({word:#x})")
 
     line = None
     if rank == 0:
@@ -482,7 +512,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("vdit", "reference"), default="vdit")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(wl.WORKLOADS))
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--reference-seconds", type=float, default=40.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", choices=("bf16", "fp8"), default="bf16",
