@@ -127,11 +127,16 @@ __global__ void __launch_bounds__(kQuantThreads, 3)
 __device__ __forceinline__ void stage_v_block(const __nv_bfloat16* __restrict__ v, __nv_bfloat16* tile, int b, int h,
                                               int H, int Skv, int t0, int n) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int i = warp; i < kQuantBlock; i += kQuantThreads / 32) {
-        uint2 x = make_uint2(0u, 0u);
-        if (i < n) x = __ldcs(reinterpret_cast<const uint2*>(v + ((static_cast<size_t>(b) * Skv + t0 + i) * H + h) * 128) + lane);
-        reinterpret_cast<uint2*>(tile + i * 128)[lane] = x;
+    constexpr int kRows = kQuantBlock / (kQuantThreads / 32);  // rows per warp, all loads in flight at once
+    uint2 x[kRows];
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+        const int i = warp + r * (kQuantThreads / 32);
+        x[r] = make_uint2(0u, 0u);
+        if (i < n) x[r] = __ldcs(reinterpret_cast<const uint2*>(v + ((static_cast<size_t>(b) * Skv + t0 + i) * H + h) * 128) + lane);
     }
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) reinterpret_cast<uint2*>(tile + (warp + r * (kQuantThreads / 32)) * 128)[lane] = x[r];
 }
 
 // One CTA (256 threads) per (b, h, block); after staging, thread d < 128 owns
