@@ -505,6 +505,61 @@ def run_merge(args):
     return 0
 
 
+def run_group(args):
+    """Time V-Smooth's Group step (k-means + stable sort) and the K/V gather at the
+    self-attention shape of the workload: C clusters seeded from evenly spaced tokens."""
+    from video_diffusion_transformer_attention_b200 import binding as vb
+    dev = torch.device("cuda", 0)
+    call = wl.WORKLOADS[args.workload].calls[0]
+    B, H, S, D = call.B, call.H, call.Skv, call.D
+    inp = wl.workload_inputs(args.workload)
+    k, v = inp["k"].to(dev), inp["v"].to(dev)
+    C = args.clusters
+    idx = torch.linspace(0, S - 1, C).long()
+    cent0 = v[:, idx].float().permute(0, 2, 1, 3).contiguous()  # [B, H, C, D]
+    res = {}
+    for iters in (0, args.group_iters):
+        for _ in range(args.warmup):
+            vb.vsmooth_group(v, cent0.clone(), iters=iters)
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.steps):
+            cent = cent0.clone()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            vb.vsmooth_group(v, cent, iters=iters)
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        res[iters] = statistics.median(ts)
+    _, perm = vb.vsmooth_group(v, cent0.clone(), iters=0)
+    for _ in range(args.warmup):
+        vb.permute_kv(k, v, perm)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        vb.permute_kv(k, v, perm)
+    e1.record()
+    torch.cuda.synchronize()
+    g_ms = e0.elapsed_time(e1) / args.steps
+    st, word = vb.vdit_get_device_status()
+    if st != vb.VDIT_OK:
+        raise SystemExit(f"device status: {vb.vdit_status_string(st)} ({word:#x})")
+    peaks, src = load_peaks()
+    nbytes = 4 * B * S * H * D * 2  # K and V read once, written once
+    gbs = nbytes / (g_ms * 1e-3) / 1e9
+    per_iter = (res[args.group_iters] - res[0]) / max(args.group_iters, 1)
+    print(json.dumps({"kernel": "vsmooth_group (assign, accumulate, finalize, sort) + permute_rows_kernel",
+                      "workload": f"{args.workload} V: B={B} H={H} S={S} D={D}, C={C}",
+                      "assign_and_sort_ms": res[0], "ms_per_lloyd_iteration": per_iter,
+                      "assign_gfma": B * H * S * C * D / 1e9,
+                      "permute_kv": {"ms": g_ms, "bytes": nbytes, "roofline": {
+                          "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                          "frac": gbs / peaks["hbm_gbs"], "peak_kind": f"{src} copy bandwidth"}}}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -519,8 +574,11 @@ def main():
                     help="bf16 attention (default) or the 8-bit path (E4M3 + V-Smooth + ExpCast-FP8)")
     ap.add_argument("--qknorm", action="store_true",
                     help="raw Q/K with the per-head RMS norm fused into the self-attention call")
-    ap.add_argument("--kernel", choices=("attention", "merge"), default="attention",
-                    help="merge: time only the LSE merge kernel (HBM roofline)")
+    ap.add_argument("--kernel", choices=("attention", "merge", "group"), default="attention",
+                    help="merge: time only the LSE merge kernel (HBM roofline); group: V-Smooth's Group step "
+                         "and the K/V gather")
+    ap.add_argument("--clusters", type=int, default=64, help="--kernel group: clusters per head")
+    ap.add_argument("--group-iters", type=int, default=1, help="--kernel group: Lloyd iterations")
     args = ap.parse_args()
     if args.path == "fp8" and args.qknorm:
         ap.error("--qknorm applies to the bf16 path only")
@@ -530,6 +588,8 @@ def main():
         return run_reference(args)
     if args.kernel == "merge":
         return run_merge(args)
+    if args.kernel == "group":
+        return run_group(args)
     return run_vdit(args)
 
 
