@@ -277,8 +277,9 @@ def run_vdit(args):
             if st != vb.VDIT_OK:
                 raise SystemExit(f"vdit_attn_fp8_plan: {vb.vdit_status_string(st)}")
             fp8_ws.append(torch.empty(need, dtype=torch.uint8, device=dev))
-    # kernels this library launches per call of the step
-    launches_per_call = [(5 if args.path == "fp8" else 1) + (1 if args.qknorm and c.name == "self" else 0)
+    # kernels of this library launched per call of the step (the 8-bit path's
+    # zeroing of its running maxima is a cudaMemsetAsync, not one of these)
+    launches_per_call = [(4 if args.path == "fp8" else 1) + (1 if args.qknorm and c.name == "self" else 0)
                          for c in w.calls]
 
     def launch(i, call, q, k, v, o, lse, mid_event=None):
