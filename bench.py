@@ -568,7 +568,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("vdit", "reference"), default="vdit")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(wl.WORKLOADS))
-    ap.add_argument("--e2e-steps", type=int, default=6)
+    ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--reference-seconds", type=float, default=40.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", choices=("bf16", "fp8"), default="bf16",
