@@ -186,12 +186,15 @@ def test_lse_is_optional():
     assert torch.equal(o1, o2)
 
 
+# 512 rows per head (every head), including the first and last rows and the
+# rows on both sides of tile and chunk boundaries; each row is computed by the
+# oracle exactly, against all of its allowed keys
 LARGE = [
-    ("wan21_1p3b_480p", 0, 48),
-    ("wan22_720p_16x16", 0, 16),
-    ("wan21_14b_720p", 0, 12),
-    ("wan21_14b_720p", 1, 48),
-    ("block_causal_7x4680", 0, 48),
+    ("wan21_1p3b_480p", 0, 512),
+    ("wan22_720p_16x16", 0, 512),
+    ("wan21_14b_720p", 0, 512),
+    ("wan21_14b_720p", 1, 512),
+    ("block_causal_7x4680", 0, 512),
 ]
 
 
