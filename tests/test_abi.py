@@ -149,6 +149,65 @@ def test_qk_rms_norm_argument_checks():
     assert call(Sq=0, Skv=0) == vb.VDIT_OK                              # nothing to do, nothing launched
 
 
+def test_fp8_entry_point_argument_checks():
+    st, parts, total = vb.vdit_fp8_layout(1, 2, 300, 333, 128)
+    assert st == vb.VDIT_OK and total > 0
+    assert list(parts.values()) == sorted(parts.values())                       # parts in order
+    assert all(o % 256 == 0 for o in parts.values())                            # each 256-byte aligned
+    assert parts["k"] - parts["q"] >= 300 * 2 * 128                             # Q codes: one byte per element
+    st, need = vb.vdit_attn_fp8_plan(1, 2, 300, 333, 128, 0, 0)
+    assert st == vb.VDIT_OK and need == total
+    assert vb.vdit_attn_fp8_plan(1, 2, 300, 333, 128, vb.VDIT_MASK_BLOCK_SPARSE, 0)[0] == vb.VDIT_ERR_INVALID_ARG
+    assert vb.vdit_attn_fp8_plan(1, 2, 300, 333, 64, 0, 0)[0] == vb.VDIT_ERR_UNSUPPORTED
+    ws = A * 64
+    q, k, v, o, lse = A, A * 3, A * 5, A * 7, A * 9
+    assert vb.vdit_fp8_quantize(q, k, v, 1, 2, 300, 333, 128, None, 0, stream=0, check=False) == vb.VDIT_ERR_WORKSPACE
+    assert vb.vdit_fp8_quantize(q, k, v, 1, 2, 300, 333, 128, ws, total - 1, stream=0,
+                                check=False) == vb.VDIT_ERR_WORKSPACE
+    assert vb.vdit_fp8_quantize(q, k, v, 1, 2, 300, 333, 128, ws + 128, total, stream=0,
+                                check=False) == vb.VDIT_ERR_MISALIGNED
+    assert vb.vdit_fp8_quantize(q, k, v + 8, 1, 2, 300, 333, 128, ws, total, stream=0,
+                                check=False) == vb.VDIT_ERR_MISALIGNED
+    assert vb.vdit_fp8_quantize(q, k, v, 1, 2, 300, 333, 128, q, total, stream=0,
+                                check=False) == vb.VDIT_ERR_INVALID_ARG           # workspace over q
+    assert vb.vdit_attn_fwd_fp8(q, k, v, o, lse, 1, 2, 300, 333, 128, 0.1, vb.VDIT_MASK_BLOCK_CAUSAL, 100, ws,
+                                total, stream=0, check=False) == vb.VDIT_ERR_INVALID_ARG   # needs Sq == Skv
+    assert vb.vdit_attn_fwd_fp8(q, k, v, o, lse, 1, 2, 300, 333, 128, -1.0, 0, 0, ws, total, stream=0,
+                                check=False) == vb.VDIT_ERR_INVALID_ARG
+    assert vb.vdit_attn_fwd_fp8_quantized(o, lse, 1, 2, 300, 333, 128, 0.1, 0, 0, ws, total - 256, stream=0,
+                                          check=False) == vb.VDIT_ERR_WORKSPACE
+
+
+def test_group_entry_point_argument_checks():
+    st, need = vb.vdit_vsmooth_group_plan(1, 2, 1000, 128, 64)
+    assert st == vb.VDIT_OK and need >= 2 * 64 * 128 * 4 + 2 * 64 * 4
+    for C in (0, 65):
+        assert vb.vdit_vsmooth_group_plan(1, 2, 1000, 128, C)[0] == vb.VDIT_ERR_INVALID_ARG
+    assert vb.vdit_vsmooth_group_plan(1, 2, 1000, 64, 8)[0] == vb.VDIT_ERR_UNSUPPORTED
+    v, cent, labels, perm, ws = A, A * 3, A * 5, A * 7, A * 64
+
+    def group(**kw):
+        a = dict(v=v, centroids=cent, labels=labels, perm=perm, iters=2, workspace=ws, nbytes=need)
+        a.update(kw)
+        return vb.vdit_vsmooth_group(a["v"], a["centroids"], a["labels"], a["perm"], 1, 2, 1000, 128, 64,
+                                     a["iters"], a["workspace"], a["nbytes"], stream=0, check=False)
+    assert group(workspace=None) == vb.VDIT_ERR_WORKSPACE
+    assert group(nbytes=need - 4) == vb.VDIT_ERR_WORKSPACE
+    assert group(labels=labels + 2) == vb.VDIT_ERR_MISALIGNED
+    assert group(iters=-1) == vb.VDIT_ERR_INVALID_ARG
+    assert group(perm=labels) == vb.VDIT_ERR_INVALID_ARG                         # labels and perm overlap
+    assert group(workspace=v) == vb.VDIT_ERR_INVALID_ARG                         # workspace over v
+    k, kout, vout = A * 9, A * 11, A * 13
+    assert vb.vdit_permute_kv(k, v, perm, kout, vout, 1, 2, 1000, 64, stream=0,
+                              check=False) == vb.VDIT_ERR_UNSUPPORTED
+    assert vb.vdit_permute_kv(k, v, perm, kout, kout, 1, 2, 1000, 128, stream=0,
+                              check=False) == vb.VDIT_ERR_INVALID_ARG             # both outputs in one buffer
+    assert vb.vdit_permute_kv(k, v, perm, k, vout, 1, 2, 1000, 128, stream=0,
+                              check=False) == vb.VDIT_ERR_INVALID_ARG             # in place is not allowed
+    assert vb.vdit_permute_kv(k, v, perm, kout + 4, vout, 1, 2, 1000, 128, stream=0,
+                              check=False) == vb.VDIT_ERR_MISALIGNED
+
+
 def test_empty_call_is_a_no_op():
     for B, H, Sq in [(0, 2, 64), (1, 0, 64), (1, 2, 0)]:
         assert vb.vdit_attn_fwd(None, None, None, None, None, B, H, Sq, 64, 128, 0.1, 0, 0,
