@@ -221,6 +221,11 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&s)[32], uint64_t scal
 
 // ---------------------------------------------------------------- kernel
 
+// kSparse: the block-sparse instantiation, whose query tiles each take part
+// only in the key tiles their own mask rows allow.  The dense, block-causal
+// and cross instantiation keeps the plain issue order, in which both tiles
+// take part in every key tile.
+template <bool kSparse>
 __global__ void __launch_bounds__(kNumThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -263,7 +268,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     }
     uint16_t* kv_list = reinterpret_cast<uint16_t*>(smem + kSmemList);
     int* kv_list_len = reinterpret_cast<int*>(smem + kSmemList + kMaxSparseKvBlocks * 2);
-    if (p.mask_kind == kMaskBlockSparse && warp == kListWarp) {
+    if (kSparse && warp == kListWarp) {
         // Compact the key blocks either query tile of this CTA attends to,
         // in ascending order, each tagged with which of the two tiles may use it.
         const int qb0 = q0 / kSparseBlock;
@@ -286,7 +291,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = bars->tmem_base;
-    const bool sparse = p.mask_kind == kMaskBlockSparse;
+    constexpr bool sparse = kSparse;
 
     // Keys this CTA needs: all of them, or for block-causal everything up to
     // the end of the chunk that holds the CTA's last valid query row.
@@ -338,6 +343,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             bool ok = n_kv > 0 &&
                       bounded_wait(smem_addr(&bars->q_full[0]), 0, abort_flag, p.timeout_ns, kSiteMma) &&
                       bounded_wait(smem_addr(&bars->q_full[1]), 0, abort_flag, p.timeout_ns, kSiteMma);
+            if constexpr (!kSparse) {
             // prologue: S_0 and S_1 against K_0
             if (ok) ok = bounded_wait(smem_addr(&bars->kv_full[0]), 0, abort_flag, p.timeout_ns, kSiteMma);
             if (ok) {
@@ -384,6 +390,73 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     }
                 }
             }
+            } else {
+            // A query tile takes part in key tile e unless a block-sparse entry
+            // leaves it out; its S and P V are then skipped, and its barrier
+            // phases count only the key tiles it takes part in.
+            auto part = [&](int e, int t) -> bool { return !sparse || ((kv_list[e] >> (14 + t)) & 1u); };
+            int last[2] = {n_kv - 1, n_kv - 1};  // each tile's last key tile (-1: none)
+            if (sparse) {
+                last[0] = last[1] = -1;
+                for (int e = n_kv - 1; e >= 0 && (last[0] < 0 || last[1] < 0); --e) {
+                    if (last[0] < 0 && part(e, 0)) last[0] = e;
+                    if (last[1] < 0 && part(e, 1)) last[1] = e;
+                }
+            }
+            int done[2] = {0, 0};  // P V products issued per tile
+            // prologue: the scores of the tiles that take part in key tile 0
+            if (ok) ok = bounded_wait(smem_addr(&bars->kv_full[0]), 0, abort_flag, p.timeout_ns, kSiteMma);
+            if (ok) {
+                tc_fence_after_sync();
+                for (int t = 0; t < kQTiles; ++t) {
+                    if (!part(0, t)) continue;
+                    issue_qk(tS[t], q_desc[t], k_desc0);
+                    umma_commit(smem_addr(&bars->s_full[t]));
+                }
+                umma_commit(smem_addr(&bars->kv_empty[0]));
+            }
+            // steady state, per key tile j (each step only for the tiles that take part):
+            //   PV0(j) [two halves]  S0(j+1)  PV1(j) [two halves]  S1(j+1)
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int uv = 2 * j + 1;
+                const int v_slot = uv % kStages;
+                const int uk = 2 * (j + 1);
+                const int k_slot = uk % kStages;
+                const bool more = (j + 1) < n_kv;
+                bool k_ready = false;
+                ok = bounded_wait(smem_addr(&bars->kv_full[v_slot]), uint32_t(uv / kStages) & 1u, abort_flag,
+                                  p.timeout_ns, kSiteMma);
+                for (int t = 0; ok && t < kQTiles; ++t) {
+                    if (part(j, t)) {
+                        const uint32_t ph = uint32_t(done[t]) & 1u;
+                        for (int hf = 0; ok && hf < 2; ++hf) {
+                            ok = bounded_wait(smem_addr(&bars->p_full[t][hf]), ph, abort_flag, p.timeout_ns,
+                                              kSiteMma);
+                            if (ok) {
+                                tc_fence_after_sync();
+                                issue_pv_half(tO[t], tS[t], v_desc0 + uint64_t(v_slot) * kSlotStep, hf, done[t] > 0);
+                            }
+                        }
+                        if (!ok) break;
+                        ++done[t];
+                        if (j == last[t]) umma_commit(smem_addr(&bars->o_full[t]));
+                    }
+                    if (t == 1) umma_commit(smem_addr(&bars->kv_empty[v_slot]));
+                    if (more && part(j + 1, t)) {
+                        if (!k_ready) {
+                            ok = bounded_wait(smem_addr(&bars->kv_full[k_slot]), uint32_t(uk / kStages) & 1u,
+                                              abort_flag, p.timeout_ns, kSiteMma);
+                            if (!ok) break;
+                            tc_fence_after_sync();
+                            k_ready = true;
+                        }
+                        issue_qk(tS[t], q_desc[t], k_desc0 + uint64_t(k_slot) * kSlotStep);
+                        umma_commit(smem_addr(&bars->s_full[t]));
+                    }
+                }
+                if (ok && more) umma_commit(smem_addr(&bars->kv_empty[k_slot]));  // after every S of K_(j+1)
+            }
+            }
             if (!ok) {
                 // Let every MMA already issued finish before TMEM is released;
                 // this wait ignores the abort flag but keeps its time limit.
@@ -417,8 +490,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         float l = 0.0f;       // running row sum at that reference
         bool ok = true;
 
+        int taken = 0;  // key tiles this query tile has taken part in
         for (int j = 0; j < n_kv; ++j) {
-            ok = warp_wait(s_full, uint32_t(j) & 1u, abort_flag, p.timeout_ns, kSiteSoftmax);
+            if (kSparse && !((kv_list[j] >> (14 + t)) & 1u)) continue;  // this tile sits this key tile out
+            const int idx = kSparse ? taken : j;  // this tile's count of key tiles so far
+            ok = warp_wait(s_full, uint32_t(idx) & 1u, abort_flag, p.timeout_ns, kSiteSoftmax);
             if (!ok) break;
             tc_fence_after_sync();
             uint32_t s[4][32];
@@ -457,8 +533,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             };
             uint64_t lsum[4] = {0, 0, 0, 0};
             uint32_t pa[2][16];  // packed P of keys 0-63, held until the reference max is settled
-            if (j == 0) {
-                // first tile: the reference max is the tile max
+            if (idx == 0) {
+                // first key tile: the reference max is the tile max
                 m = tile_max() * scale_log2;
                 const float m_use = (m == -INFINITY) ? 0.0f : m;
                 const uint64_t negm2 = pack_f32x2(-m_use, -m_use);
@@ -529,11 +605,14 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     part += __uint_as_float(uint32_t(lsum[q])) + __uint_as_float(uint32_t(lsum[q] >> 32));
                 l += part;
             }
+            if (kSparse) ++taken;
         }
 
-        // With no key tile at all (an empty block-sparse list) O stays 0 and
-        // LSE = -inf; nothing was issued, so there is nothing to wait for.
-        if (ok && n_kv > 0) ok = warp_wait(smem_addr(&bars->o_full[t]), 0, abort_flag, p.timeout_ns, kSiteSoftmax);
+        // With no key tile for this query tile (nothing it attends to in a
+        // block-sparse mask) O stays 0 and LSE = -inf; nothing was issued for
+        // it, so there is nothing to wait for.
+        const int n_mine = kSparse ? taken : n_kv;  // key tiles this query tile took part in
+        if (ok && n_mine > 0) ok = warp_wait(smem_addr(&bars->o_full[t]), 0, abort_flag, p.timeout_ns, kSiteSoftmax);
         if (ok) {
             tc_fence_after_sync();
             const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
@@ -541,7 +620,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t o[32];
-                if (n_kv > 0) {
+                if (n_mine > 0) {
                     tmem_ld32(tO + uint32_t(c) * 32u, o);
                     tmem_ld_wait(o);
                 } else {

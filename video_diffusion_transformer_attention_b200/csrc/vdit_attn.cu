@@ -76,7 +76,9 @@ void init_device(int dev, DeviceState* st) {
         st->status = VDIT_ERR_UNSUPPORTED;
         return;
     }
-    if (cudaFuncSetAttribute(vdit::attn_fwd_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(vdit::attn_fwd_sm100_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             vdit::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(vdit::attn_fwd_sm100_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              vdit::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(vdit::attn_fwd_fp8_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              vdit::kF8SmemBytes) != cudaSuccess) {
@@ -169,7 +171,10 @@ vdit_status launch(const void* q, const void* k, const void* v, void* o, float* 
     p.n_kvb = (s.Skv + vdit::kSparseBlock - 1) / vdit::kSparseBlock;
     dim3 grid(grid_x(s.Sq), s.H, s.B);
     if (!after_norm) {
-        vdit::attn_fwd_sm100_kernel<<<grid, vdit::kNumThreads, vdit::kSmemBytes, stream>>>(tq, tk, tv, p);
+        if (s.mask_kind == VDIT_MASK_BLOCK_SPARSE)
+            vdit::attn_fwd_sm100_kernel<true><<<grid, vdit::kNumThreads, vdit::kSmemBytes, stream>>>(tq, tk, tv, p);
+        else
+            vdit::attn_fwd_sm100_kernel<false><<<grid, vdit::kNumThreads, vdit::kSmemBytes, stream>>>(tq, tk, tv, p);
         return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
     }
     // Programmatic dependent of the Q/K norm kernel just queued on this
@@ -185,8 +190,9 @@ vdit_status launch(const void* q, const void* k, const void* v, void* o, float* 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, vdit::attn_fwd_sm100_kernel, tq, tk, tv, p) == cudaSuccess ? VDIT_OK
-                                                                                             : VDIT_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, vdit::attn_fwd_sm100_kernel<false>, tq, tk, tv, p) == cudaSuccess
+               ? VDIT_OK
+               : VDIT_ERR_CUDA;
 }
 
 vdit_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
