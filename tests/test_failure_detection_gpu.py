@@ -54,6 +54,33 @@ def test_withheld_kv_times_out_and_context_survives():
     assert res["ok"], res
 
 
+def test_cross_attention_over_several_waves_times_out_and_context_survives():
+    """More CTAs than SMs: later waves start after the first ones gave up."""
+    dev = torch.device("cuda:0")
+    B, H, Sq, Skv, D = 1, 8, 20000, 512, 128
+    q, k, v = wl.draw_qkv(B, H, Sq, Skv, D, seed=33, recipe="rms_qk")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    o = torch.empty_like(qd)
+    lse = torch.empty((B, H, Sq), dtype=torch.float32, device=dev)
+    assert vb.vdit_get_device_status()[0] == vb.VDIT_OK
+    st = vb.vdit_testing_attn_fwd(qd, kd, vd, o, lse, B, H, Sq, Skv, D, 1 / math.sqrt(D), vb.VDIT_MASK_CROSS, 0,
+                                  vb.VDIT_TESTING_WITHHOLD_KV, 100_000_000)
+    assert st == vb.VDIT_OK
+    st, word = vb.vdit_get_device_status()
+    assert st == vb.VDIT_ERR_TIMEOUT
+    assert word & 1 and word & SITE_MMA
+    assert vb.vdit_get_device_status() == (vb.VDIT_OK, 0)
+    o2, lse2 = vb.attention(qd, kd, vd, 1 / math.sqrt(D), vb.VDIT_MASK_CROSS, 0)
+    assert vb.vdit_get_device_status()[0] == vb.VDIT_OK
+    rows = np.array([0, 1, 255, 256, 9999, 19744, 19999])
+    o_r, l_r = oracle_attention(wl.bf16_bits(q[:, rows]), wl.bf16_bits(k), wl.bf16_bits(v), 1 / math.sqrt(D))
+    o_g = o2.float().cpu().numpy().astype(np.float64)[:, rows]
+    l_g = lse2.cpu().numpy().astype(np.float64)[:, :, rows]
+    res = check_parity(o_g[0].transpose(1, 0, 2).reshape(-1, D), o_r[0].transpose(1, 0, 2).reshape(-1, D),
+                       l_g.reshape(-1), l_r.reshape(-1), None, "cross, after timeout")
+    assert res["ok"], res
+
+
 def test_testing_entry_point_without_fault_matches_the_product_call():
     dev = torch.device("cuda:0")
     B, H, S, D = 1, 2, 700, 128

@@ -87,6 +87,35 @@ def test_parity_all_rows(B, H, Sq, Skv, mask, chunk, recipe):
     compare_all_rows(q, k, v, 1 / math.sqrt(128), mask, chunk, f"{B}x{H}x{Sq}x{Skv} m{mask} c{chunk}")
 
 
+# Cross attention with more CTAs (256 query rows of one head each) than SMs,
+# every row compared: short text sequences of one to four key tiles, ragged
+# query and key tails, batch > 1.
+WIDE_CROSS = [
+    # B, H, Sq, Skv
+    (2, 5, 9000, 77),      # one key tile
+    (1, 4, 20000, 300),    # three key tiles, ragged query and key tails
+    (1, 40, 9000, 130),    # about ten waves of CTAs, two key tiles
+    (1, 3, 30000, 512),    # the text length of the 720p workload
+]
+
+
+@pytest.mark.parametrize("B,H,Sq,Skv", WIDE_CROSS)
+def test_cross_attention_over_several_waves(B, H, Sq, Skv):
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert B * H * -(-Sq // 256) > sms  # more CTAs than SMs
+    q, k, v = wl.draw_qkv(B, H, Sq, Skv, 128, seed=41 + Sq + Skv, recipe="rms_qk")
+    compare_all_rows(q, k, v, 1 / math.sqrt(128), CROSS, 0, f"cross {B}x{H}x{Sq}x{Skv}")
+
+
+def test_cross_attention_is_deterministic():
+    dev = torch.device("cuda:0")
+    q, k, v = (t.to(dev) for t in wl.draw_qkv(1, 8, 20000, 512, 128, seed=42, recipe="rms_qk"))
+    o1, l1 = vb.attention(q, k, v, None, CROSS, 0)
+    o2, l2 = vb.attention(q, k, v, None, CROSS, 0)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
 def test_parity_other_scales():
     q, k, v = wl.draw_qkv(1, 2, 400, 400, 128, seed=3, recipe="iid")
     for scale in (0.02, 0.2):

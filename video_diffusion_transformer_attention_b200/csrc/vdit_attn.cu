@@ -47,7 +47,10 @@ vdit_status check_shape(const Shape& s, bool check_scale, float scale) {
     return VDIT_OK;
 }
 
-int grid_x(int Sq) { return (Sq + vdit::kQTiles * vdit::kBlockM - 1) / (vdit::kQTiles * vdit::kBlockM); }
+int grid_x(int Sq) {
+    const long long rows = vdit::kQTiles * vdit::kBlockM;  // query rows per CTA; no int overflow near INT_MAX
+    return static_cast<int>((static_cast<long long>(Sq) + rows - 1) / rows);
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
