@@ -58,7 +58,11 @@ typedef enum {
      * Sq == Skv.  Keys of later chunks are skipped, not just masked. */
     VDIT_MASK_BLOCK_CAUSAL = 1,
     /* Same arithmetic as FULL; the caller says the keys are a short text
-     * sequence (Skv << Sq), e.g. 512 text tokens. */
+     * sequence (Skv << Sq), e.g. 512 text tokens, and the launch takes the
+     * short-key schedule: persistent CTAs, two per SM, each taking one
+     * 128-row query tile at a time and loading the next tile's Q while it
+     * finishes the current one.  Any Skv is correct; long key sequences run
+     * faster as FULL. */
     VDIT_MASK_CROSS = 2,
     /* A(i) = { j : mask[b][h][i / 128][j / 128] != 0 }, a caller-given byte
      * per (128-query, 128-key) block pair; key blocks no query of a tile pair
@@ -86,8 +90,10 @@ typedef enum {
  * vdit_attn_plan -- host-only query, touches no device.
  * Writes the workspace size the _ws entry point needs (0 for every shape in
  * this version) and, if grid_ctas is non-NULL, the number of CTAs the
- * forward launches.  Same argument rules as vdit_attn_fwd, except that
- * pointers are not involved.
+ * forward launches: B * H * ceil(Sq / 256), or for CROSS the number of
+ * 128-row query tiles, B * H * ceil(Sq / 128), which the launch shares out
+ * over at most two persistent CTAs per SM.  Same argument rules as
+ * vdit_attn_fwd, except that pointers are not involved.
  */
 vdit_status vdit_attn_plan(int B, int H, int Sq, int Skv, int D, int mask_kind,
                            int chunk_tokens, size_t* workspace_bytes,

@@ -49,6 +49,9 @@ def test_plan_reports_grid_and_zero_workspace():
     assert ws == 0 and grid == 296 * 40
     ws, grid = vb.vdit_attn_plan(2, 3, 300, 300, 128, vb.VDIT_MASK_BLOCK_CAUSAL, 100)
     assert grid == 2 * 3 * 2
+    # cross attention: one 128-row query tile per CTA
+    ws, grid = vb.vdit_attn_plan(1, 40, 75600, 512, 128, vb.VDIT_MASK_CROSS, 0)
+    assert ws == 0 and grid == 591 * 40
     assert vb.vdit_attn_plan(1, 1, 0, 5, 128, 0, 0) == (0, 0)
 
 

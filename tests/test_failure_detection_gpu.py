@@ -55,7 +55,7 @@ def test_withheld_kv_times_out_and_context_survives():
 
 
 def test_cross_attention_over_several_waves_times_out_and_context_survives():
-    """More CTAs than SMs: later waves start after the first ones gave up."""
+    """The persistent cross launch: every CTA holds several query tiles when the wait runs out."""
     dev = torch.device("cuda:0")
     B, H, Sq, Skv, D = 1, 8, 20000, 512, 128
     q, k, v = wl.draw_qkv(B, H, Sq, Skv, D, seed=33, recipe="rms_qk")

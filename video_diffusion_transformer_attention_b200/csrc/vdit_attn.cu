@@ -15,6 +15,7 @@
 #include "vdit_attn.h"
 #include "vdit_attn_testing.h"
 #include "attn_fwd_sm100.cuh"
+#include "attn_cross_sm100.cuh"
 #include "attn_merge.cuh"
 #include "qk_norm.cuh"
 #include "fp8_quant.cuh"
@@ -52,6 +53,9 @@ int grid_x(int Sq) {
     return static_cast<int>((static_cast<long long>(Sq) + rows - 1) / rows);
 }
 
+// 128-row query tiles per (batch, head): the cross-attention work items
+int cross_tiles(int Sq) { return static_cast<int>((static_cast<long long>(Sq) + vdit::kBlockM - 1) / vdit::kBlockM); }
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
@@ -64,7 +68,8 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 struct DeviceState {
     std::once_flag once;
     vdit_status status = VDIT_ERR_CUDA;
-    int norm_grid = 0;  // one full wave of qk_rms_norm_kernel blocks
+    int norm_grid = 0;   // one full wave of qk_rms_norm_kernel blocks
+    int cross_grid = 0;  // the persistent cross-attention grid: two CTAs per SM
 };
 DeviceState g_devices[kMaxDevices];
 
@@ -83,6 +88,11 @@ void init_device(int dev, DeviceState* st) {
                              vdit::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(vdit::attn_fwd_sm100_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              vdit::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(vdit::attn_cross_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             vdit::kCrossSmemBytes) != cudaSuccess ||
+        // all of the unified L1 / shared storage as shared memory: two CTAs fit
+        cudaFuncSetAttribute(vdit::attn_cross_sm100_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
         cudaFuncSetAttribute(vdit::attn_fwd_fp8_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              vdit::kF8SmemBytes) != cudaSuccess) {
         st->status = VDIT_ERR_CUDA;
@@ -97,6 +107,12 @@ void init_device(int dev, DeviceState* st) {
         return;
     }
     st->norm_grid = sms * per_sm;
+    // Two CTAs per SM: what the cross kernel's TMEM (256 of 512 columns),
+    // registers (2 x 192 x 168) and shared memory (2 x 97 KB) allow.  The
+    // occupancy query reports one for this kernel, but two run side by side
+    // (measured: 1.02 vs 1.68 ms at Sq = 75,600, H = 40, Skv = 512).  The CTAs
+    // never wait on one another, so the grid is correct at any residency.
+    st->cross_grid = sms * 2;
     st->status = VDIT_OK;
 }
 
@@ -151,7 +167,8 @@ vdit_status launch(const void* q, const void* k, const void* v, void* o, float* 
                    const Shape& s, float scale, int debug_flags, unsigned long long timeout_ns, cudaStream_t stream,
                    bool after_norm) {
     int dev = 0;
-    vdit_status st = ensure_device(&dev);
+    const DeviceState* ds = nullptr;
+    vdit_status st = ensure_device(&dev, &ds);
     if (st != VDIT_OK) return st;
     CUtensorMap tq, tk, tv;
     if (!encode_bshd(&tq, q, s.B, s.Sq, s.H) || !encode_bshd(&tk, k, s.B, s.Skv, s.H) ||
@@ -172,6 +189,27 @@ vdit_status launch(const void* q, const void* k, const void* v, void* o, float* 
     p.block_mask = block_mask;
     p.n_qb = (s.Sq + vdit::kSparseBlock - 1) / vdit::kSparseBlock;
     p.n_kvb = (s.Skv + vdit::kSparseBlock - 1) / vdit::kSparseBlock;
+    if (s.mask_kind == VDIT_MASK_CROSS) {
+        // Short key sequence: persistent, two CTAs per SM, one 128-row query tile per item.
+        const long long items = static_cast<long long>(p.n_qb) * s.H * s.B;
+        const dim3 grid(static_cast<unsigned>(items < ds->cross_grid ? items : ds->cross_grid));
+        if (!after_norm) {
+            vdit::attn_cross_sm100_kernel<<<grid, vdit::kCrossThreads, vdit::kCrossSmemBytes, stream>>>(tq, tk, tv, p);
+            return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
+        }
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(vdit::kCrossThreads);
+        cfg.dynamicSmemBytes = vdit::kCrossSmemBytes;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, vdit::attn_cross_sm100_kernel, tq, tk, tv, p) == cudaSuccess ? VDIT_OK
+                                                                                                     : VDIT_ERR_CUDA;
+    }
     dim3 grid(grid_x(s.Sq), s.H, s.B);
     if (!after_norm) {
         if (s.mask_kind == VDIT_MASK_BLOCK_SPARSE)
@@ -502,7 +540,8 @@ vdit_status vdit_attn_plan(int B, int H, int Sq, int Skv, int D, int mask_kind, 
         if (workspace_bytes == nullptr) return VDIT_ERR_INVALID_ARG;
         *workspace_bytes = 0;
         if (grid_ctas != nullptr) {
-            const long long n = (B == 0 || H == 0 || Sq == 0) ? 0 : (long long)grid_x(Sq) * H * B;
+            const long long per_bh = mask_kind == VDIT_MASK_CROSS ? cross_tiles(Sq) : grid_x(Sq);
+            const long long n = (B == 0 || H == 0 || Sq == 0) ? 0 : per_bh * H * B;
             *grid_ctas = n > 0x7fffffffLL ? 0x7fffffff : int(n);
         }
         return VDIT_OK;
