@@ -17,12 +17,14 @@ Shapes come from the pages' Wan-style workloads:
 * Value outliers concentrated in a few channels that differ between heads --
   "VC-Attention" (aikraft.ru), section 02 "V-Smooth".
 
-Recipe (see the design doc for the readings): a CPU ``torch.Generator`` seeded with
+Recipe (the pages give shapes and value statistics but no generator, so the
+choices below are this module's): a CPU ``torch.Generator`` seeded with
 ``1000 + config index`` draws Q, K, V (in that order) as N(0, 1) float32 in
 [B, S, H, D] layout.  Where a workload says so, Q and K are RMS-normalised over
 each (token, head) D-vector in float32 (``x / sqrt(mean(x^2) + 1e-6)``, weight
 1), and 3 of the 128 V channels of each head -- picked by a seeded permutation
-per head -- are multiplied by 8.  Everything is then rounded to bf16, and those
+per head (round(2% of 128) = 3; the gain 8 is exact in bf16) -- are multiplied
+by 8.  Everything is then rounded to bf16, and those
 bf16 values are the inputs.  Cross-attention text K/V come from a second
 generator seeded ``2000 + config index``.
 """
