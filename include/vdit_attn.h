@@ -214,7 +214,14 @@ vdit_status vdit_attn_fwd_qknorm(const void* q, const void* k, const void* v,
  *
  * The first call on a device looks up the scratch's device address (once
  * per device, with that device current); make that first call before any
- * stream capture.  All calls on a device share the one scratch buffer and it
+ * stream capture.  Only a lookup that succeeded is kept, so a first call
+ * that failed is retried by the next one.  The address stays valid until the
+ * device is reset (cudaDeviceReset unloads the library's device code, as it
+ * does the kernel attributes the library sets once per device); do not reset
+ * a device while the library is in use on it.  Arguments are checked in the
+ * order vdit_attn_fwd_qknorm checks them, so both accept the same calls; on
+ * a GPU that is not sm_100 the call returns VDIT_ERR_UNSUPPORTED.
+ * All calls on a device share the one scratch buffer and it
  * keeps the last call's contents (nothing in it needs to start at zero), so
  * calls whose work overlaps on the GPU (other streams, or other host threads
  * without ordering between their streams) race on it: order them.
@@ -362,6 +369,22 @@ vdit_status vdit_attn_fwd_ws(const void* q, const void* k, const void* v,
 vdit_status vdit_attn_merge(void* o_acc, float* lse_acc, const void* o_part,
                             const float* lse_part, int B, int H, int S, int D,
                             void* stream);
+
+/*
+ * vdit_attn_merge_f32 -- vdit_attn_merge with the running O kept in fp32.
+ * Same formula and rules, but o_acc is device fp32 [B][S][H][D], so a ring
+ * of N ranks rounds its merged O to bf16 once instead of after each of its
+ * N - 1 folds.  o_part stays bf16 (the forward's output).  o_out, when not
+ * NULL, is a device bf16 [B][S][H][D] buffer that also receives the merged O
+ * rounded to bf16 (round to nearest even); pass it on the last fold.
+ * Start a ring with o_acc = 0 and lse_acc = -inf: the first fold then copies
+ * the first partial exactly.  No buffer may overlap another except o_acc and
+ * lse_acc with themselves; pointers 16-byte aligned.  Asynchronous on
+ * `stream`.  The same passages define it as vdit_attn_merge.
+ */
+vdit_status vdit_attn_merge_f32(float* o_acc, float* lse_acc, const void* o_part,
+                                const float* lse_part, void* o_out, int B,
+                                int H, int S, int D, void* stream);
 
 /*
  * vdit_get_device_status -- synchronises `stream`, then reads and clears the

@@ -24,6 +24,14 @@ integer; the reference is raised when a tile's max exceeds it by more than
 RESCALE_CODES; the per-channel V scale is shared by all blocks of a head and
 floored at 2^-8 of the largest block mean.
 
+Two statements of the attention are given.  ``attention_fp8_plain`` is the
+page's ExpCast as stated: every byte against its row's true maximum, no
+tiles, no running reference -- the independent check of the kernel's
+attention.  ``attention_fp8`` walks the keys in 128-key tiles with a lazily
+raised reference on a grid, the schedule the kernel uses, so that the
+kernel's probability bytes can be checked one for one as a second, tighter
+test; it is not an independent statement of the method.
+
 Where floating point decides a stored code (the quantised Q, K, V and the
 scales), this module uses the same fp32 operations as the kernel, so those
 codes must match bit for bit.  The attention itself is computed in float64
@@ -185,6 +193,15 @@ def reference_for(zmax: float) -> float:
     return math.ceil(zmax - _OFFSET_FRAC) + _OFFSET_FRAC
 
 
+def expcast_row(z) -> np.ndarray:
+    """ExpCast-FP8 bytes of one row of logits z (code units, 8 x log2; -inf
+    where masked), taken against the row's own maximum, with no tiling:
+    byte_j = rint(z_j - max z + CODE_OFFSET), clamped below at 0.  The largest
+    logit gets rint(95.65) = 96, the byte of 2^P_SHIFT."""
+    z = np.asarray(z, dtype=np.float64)
+    return expcast_codes(z - z.max())
+
+
 def _allowed_prefix(mask_kind, i, Skv, chunk):
     if mask_kind == MASK_BLOCK_CAUSAL:
         return min(Skv, (i // chunk + 1) * chunk)
@@ -259,3 +276,76 @@ def attention_fp8(q_bits, k_bits, v_bits, scale: float, mask_kind: int = MASK_FU
         o_full[b, i, h] = o[r]
         lse_full[b, h, i] = lse[r]
     return o_full, lse_full
+
+
+def attention_fp8_plain(q_bits, k_bits, v_bits, scale: float, mask_kind: int = MASK_FULL, chunk_tokens: int = 0,
+                        rows=None, quantized=None, spread: bool = False):
+    """The 8-bit attention with ExpCast-FP8 as the VC-Attention page states it:
+    every probability byte is taken against its row's true maximum.
+
+    This is the plain statement of section 03 ("ExpCast-FP8") on the operands
+    of section 02 ("V-Smooth"), without any of a kernel's scheduling choices:
+    no 128-key tiles, no lazily raised running reference, no reference grid.
+    For each query row i of (b, h), over all of its allowed keys j at once:
+      z_j    = 8 log2(e) scale sq sk_j (q_codes . k_codes_j)   (code units)
+      byte_j = expcast_row(z)_j = rint(z_j - max z + 95.65), clamped at 0
+      p_j    = value(byte_j) / 2^P_SHIFT       (2^P_SHIFT: reading of the page's range)
+      v^_j   = value(code_v_j) scale_v + mu_block(j)   (V-Smooth's Demean undone: Restore)
+    O = sum_j p_j v^_j / sum_j p_j,  LSE = ln 2 (max z / 8 + log2 sum_j p_j).
+    The only readings it shares with attention_fp8 are those of the operands
+    (E4M3 blocks, V-Smooth's scales) and of the byte map (P_SHIFT, beta).
+
+    spread=True also returns, per row and head dim, sqrt(sum_j w_j^2 (v^_jd - O_d)^2)
+    with w_j = p_j / sum p -- the size of the O perturbation that independent
+    relative errors of one unit in the probabilities would cause -- and per
+    row sqrt(sum_j w_j^2), its counterpart for LSE.
+    Returns (O, LSE[, spread_o, spread_lse]) shaped like attention_fp8.
+    """
+    if quantized is None:
+        quantized = (quantize_qk(q_bits), quantize_qk(k_bits), vsmooth(v_bits))
+    (qc, qs), (kc, ks), vs = quantized
+    B, Sq, H, D = qc.shape
+    Skv = kc.shape[1]
+    if mask_kind not in (MASK_FULL, MASK_BLOCK_CAUSAL, MASK_CROSS):
+        raise ValueError("mask kind")
+    if mask_kind == MASK_BLOCK_CAUSAL and chunk_tokens < 1:
+        raise ValueError("chunk_tokens")
+    qv = e4m3_values(qc)
+    kv = e4m3_values(kc)
+    blk = np.arange(Skv) // BLOCK
+    v_hat = (e4m3_values(vs["codes"]) * vs["scale"].astype(np.float64)[:, None, :, :]
+             + vs["mu"].astype(np.float64)[:, :, blk, :].transpose(0, 2, 1, 3))          # [B, Skv, H, D]
+    if rows is None:
+        sel = [(b, h, i) for b in range(B) for h in range(H) for i in range(Sq)]
+    else:
+        sel = [tuple(int(t) for t in r) for r in np.asarray(rows).reshape(-1, 3)]
+    o = np.zeros((len(sel), D))
+    lse = np.zeros(len(sel))
+    spr = np.zeros((len(sel), D)) if spread else None
+    spl = np.zeros(len(sel)) if spread else None
+    c0 = 8.0 * LOG2E * float(scale)
+    for r, (b, h, i) in enumerate(sel):
+        n = _allowed_prefix(mask_kind, i, Skv, chunk_tokens)
+        a = c0 * float(qs[b, h, i // BLOCK]) * ks[b, h, blk[:n]].astype(np.float64)
+        z = a * (kv[b, :n, h, :] @ qv[b, i, h, :])
+        p = e4m3_values(expcast_row(z)) * 2.0 ** -P_SHIFT
+        ell = float(p.sum())
+        o[r] = p @ v_hat[b, :n, h, :] / ell
+        lse[r] = math.log(2.0) * (float(z.max()) / 8.0 + math.log2(ell))
+        if spread:
+            w = p / ell
+            spr[r] = np.sqrt((w[:, None] ** 2 * (v_hat[b, :n, h, :] - o[r]) ** 2).sum(axis=0))
+            spl[r] = math.sqrt(float((w ** 2).sum()))
+    if rows is not None:
+        return (o, lse, spr, spl) if spread else (o, lse)
+    o_full = np.zeros((B, Sq, H, D))
+    lse_full = np.zeros((B, H, Sq))
+    spr_full = np.zeros((B, Sq, H, D)) if spread else None
+    spl_full = np.zeros((B, H, Sq)) if spread else None
+    for r, (b, h, i) in enumerate(sel):
+        o_full[b, i, h] = o[r]
+        lse_full[b, h, i] = lse[r]
+        if spread:
+            spr_full[b, i, h] = spr[r]
+            spl_full[b, h, i] = spl[r]
+    return (o_full, lse_full, spr_full, spl_full) if spread else (o_full, lse_full)

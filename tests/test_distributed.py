@@ -100,12 +100,14 @@ def _fake_attn(q, k, v):
     return o, lse
 
 
-def _fake_merge(o_acc, lse_acc, o_part, lse_part):
+def _fake_merge(o_acc, lse_acc, o_part, lse_part, o_out=None):
     lse = torch.logaddexp(lse_acc, lse_part)
-    wa = torch.exp(lse_acc - lse).permute(0, 2, 1)[..., None]
+    wa = torch.nan_to_num(torch.exp(lse_acc - lse)).permute(0, 2, 1)[..., None]
     wp = torch.exp(lse_part - lse).permute(0, 2, 1)[..., None]
     o_acc.copy_(wa * o_acc + wp * o_part)
     lse_acc.copy_(lse)
+    if o_out is not None:
+        o_out.copy_(o_acc)
 
 
 def _ring_worker(rank, world, port, out):
@@ -201,3 +203,59 @@ def test_a_departed_rank_makes_the_ring_fail_instead_of_hang():
     assert out[1] == "left"
     assert out[0].startswith("error after"), out[0]
     assert float(out[0].split()[2][:-2]) < 60
+
+
+# ---------------------------------------------------------------- one problem split by heads (bench --shard heads)
+
+def _heads_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import bench
+    from video_diffusion_transformer_attention_b200 import flops as fl
+    from video_diffusion_transformer_attention_b200 import workloads as wl
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        res = {}
+        for H in (40, 12, 5):
+            h0, h1 = bench.head_range(H, world, rank)
+            got = [None] * world
+            dist.all_gather_object(got, (h0, h1))
+            res[H] = got
+        # this rank's share of the 720p workload's FLOPs, summed over the ranks
+        w = wl.WORKLOADS["wan21_14b_720p"]
+        h0, h1 = bench.head_range(w.calls[0].H, world, rank)
+        ws, _ = bench.shard_heads(w, {}, h0, h1)
+        mine = torch.tensor([sum(fl.attn_flops(c) for c in ws.calls)], dtype=torch.float64)
+        dist.all_reduce(mine)
+        res["flops"] = float(mine.item())
+        # the slices hold exactly this rank's heads
+        t = torch.arange(7, dtype=torch.float32).view(1, 1, 7, 1).expand(2, 3, 7, 4).contiguous()
+        m = torch.arange(7, dtype=torch.uint8).view(1, 7, 1, 1).expand(2, 7, 3, 3).contiguous()
+        h0, h1 = bench.head_range(7, world, rank)
+        _, sl = bench.shard_heads(wl.WORKLOADS["pr1_s1024"], {"q": t, "block_mask": m}, h0, h1)
+        res["slice"] = (sl["q"][0, 0, :, 0].tolist(), sl["block_mask"][0, :, 0, 0].tolist(),
+                        sl["q"].is_contiguous(), list(range(h0, h1)))
+        out[rank] = res
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_split_covers_every_head_once_and_counts_the_whole_problem():
+    sys.path.insert(0, ROOT)
+    from video_diffusion_transformer_attention_b200 import flops as fl
+    from video_diffusion_transformer_attention_b200 import workloads as wl
+    out = _spawn(_heads_worker)
+    for H in (40, 12, 5):
+        ranges = out[0][H]
+        assert ranges == out[1][H]
+        covered = [h for a, b in ranges for h in range(a, b)]
+        assert covered == list(range(H)), (H, ranges)
+    assert out[0][40] == [(0, 20), (20, 40)]
+    whole = sum(fl.attn_flops(c) for c in wl.WORKLOADS["wan21_14b_720p"].calls)
+    assert out[0]["flops"] == whole and out[1]["flops"] == whole
+    for rank in (0, 1):
+        q_heads, m_heads, contiguous, want = out[rank]["slice"]
+        assert q_heads == want and m_heads == want and contiguous
+    # strong-scaling throughput: the whole problem's FLOPs over the slowest rank's time
+    import bench
+    assert abs(bench.job_tflops(1, whole, 2, 100.0) - whole * 2 / 0.1 / 1e12) < 1e-9

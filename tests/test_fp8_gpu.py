@@ -1,10 +1,17 @@
 """The 8-bit path (E4M3 + V-Smooth + ExpCast-FP8) on the GPU against its oracle.
 
 The preprocessing writes integer codes and fp32 scales that the oracle
-computes with the same fp32 operations: those must match bit for bit.  The
-attention's probability bytes depend on the fp32 scores out of the tensor
-core, which can round a tie differently from the oracle's float64 scores, so
-the attention is compared with the parity bars the bf16 path uses.
+computes with the same fp32 operations: those must match bit for bit.
+
+The attention is checked twice.  Against the plain statement of ExpCast
+(oracle.fp8_oracle.attention_fp8_plain: every probability byte against its
+row's true maximum, no tiles, no running reference), under the bars derived
+in tests/helpers.py from the byte map's own log error -- the independent
+check.  And against attention_fp8, which walks the keys in the kernel's
+schedule, under the bf16 path's parity bars -- a tighter check that the
+kernel's bytes are the ones its schedule defines (they can differ by one
+code where the tensor core's fp32 scores round a tie differently from the
+oracle's float64 ones).
 """
 import math
 
@@ -14,7 +21,7 @@ import torch
 
 from oracle import attention as exact_attention
 from oracle import fp8_oracle as f8
-from tests.helpers import check_parity
+from tests.helpers import check_expcast_parity, check_parity
 from video_diffusion_transformer_attention_b200 import binding as vb
 from video_diffusion_transformer_attention_b200 import workloads as wl
 from video_diffusion_transformer_attention_b200.build import build
@@ -111,6 +118,21 @@ def test_fp8_attention_matches_its_oracle(B, H, Sq, Skv, mask, chunk, recipe):
     assert res["ok"], res
 
 
+@pytest.mark.parametrize("B,H,Sq,Skv,mask,chunk,recipe", CASES)
+def test_fp8_attention_matches_the_plain_expcast_statement(B, H, Sq, Skv, mask, chunk, recipe):
+    q, k, v = wl.draw_qkv(B, H, Sq, Skv, 128, seed=92 + Sq + Skv, recipe=recipe)
+    scale = 1 / math.sqrt(128)
+    o, lse = _run_fp8(q, k, v, mask, chunk, scale)
+    o_p, l_p, s_o, s_l = f8.attention_fp8_plain(wl.bf16_bits(q), wl.bf16_bits(k), wl.bf16_bits(v), scale, mask,
+                                                 chunk, spread=True)
+    og, lg = _flat(o, lse, B, H)
+    op, lp = _flat(o_p, l_p, B, H)
+    so, sl = _flat(s_o, s_l, B, H)
+    groups = [np.arange(i * Sq, (i + 1) * Sq) for i in range(B * H)]
+    res = check_expcast_parity(og, op, lg, lp, so, sl, groups, f"fp8 plain {B}x{H}x{Sq}x{Skv} m{mask}")
+    assert res["ok"], res
+
+
 def test_fp8_attention_with_a_wide_logit_span_takes_the_exact_clamp_and_matches():
     # Q and K x30: |logit| reaches the thousands of code units, beyond what the
     # 16-bit clamp may handle, so every warp runs the float-clamp loop
@@ -168,4 +190,10 @@ def test_fp8_attention_sampled_rows_at_a_wan_shape():
     og = np.stack([o[b, i, h] for b, h, i in rows])
     lg = np.array([lse[b, h, i] for b, h, i in rows])
     res = check_parity(og, o_r, lg, l_r, None, f"fp8 {name} sampled")
+    assert res["ok"], res
+    # the same rows against the plain ExpCast statement
+    o_p, l_p, s_o, s_l = f8.attention_fp8_plain(None, None, None, call.scale, call.mask_kind, call.chunk_tokens,
+                                                 rows=rows, quantized=quant, spread=True)
+    groups = [np.nonzero(rows[:, 1] == h)[0] for h in range(call.H)]
+    res = check_expcast_parity(og, o_p, lg, l_p, s_o, s_l, groups, f"fp8 plain {name} sampled")
     assert res["ok"], res

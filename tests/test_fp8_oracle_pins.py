@@ -249,3 +249,128 @@ def test_fp8_attention_error_splits_into_expcast_and_quantisation(mask, chunk, s
     o, l = attention(_bits(q), _bits(k), _bits(v), scale, mask, chunk)
     assert _rel(o8, o) < 0.10
     assert (np.abs(l8 - l) / np.maximum(np.abs(l), 1)).max() < 0.03
+
+
+# ------------------------------------------------------------------ the plain ExpCast statement
+
+def test_plain_expcast_row_matches_the_page_figures():
+    """Row bytes against the row's own max: in one doubling of the value range,
+    79.6% equal the bytes of exp-then-cast and none is more than one code off."""
+    gv = golden()
+    u = np.linspace(-16.0, -8.0, 1_000_001)[:-1]          # code units below the max: values 2^3 .. 2^4
+    z = np.concatenate([[0.0], u]) + 123.25               # any offset: only z - max z matters
+    bytes_ = f8.expcast_row(z).astype(int)[1:]
+    cast = torch_e4m3(np.exp2(u / 8.0 + f8.P_SHIFT)).astype(int)
+    d = bytes_ - cast
+    assert abs((d == 0).mean() * 100 - gv["match_percent"]) < 0.05
+    assert np.abs(d).max() == gv["max_code_difference"]
+    assert f8.expcast_row(np.array([3.0, 3.0, -np.inf]))[:2].tolist() == [96, 96]   # the max: 2^P_SHIFT
+    assert f8.expcast_row(np.array([0.0, -np.inf]))[1] == 0
+
+
+def test_plain_expcast_row_total_variation_stays_under_the_page_bound():
+    bound = golden()["row_tv_bound_percent"] / 100
+    g = np.random.default_rng(12)
+    worst = 0.0
+    for sigma in (0.3, 1.0, 2.0):
+        for _ in range(200):
+            x = g.standard_normal(700) * sigma               # log2-domain logits
+            c = f8.expcast_row(8.0 * x)
+            if c.min() < 8:                                  # underflow tail: outside the bound
+                continue
+            p = f8.e4m3_values(c)
+            e = np.exp2(x - x.max())
+            tv = 0.5 * np.abs(p / p.sum() - e / e.sum()).sum()
+            worst = max(worst, tv)
+    assert 0.0 < worst < bound
+
+
+def test_log_error_spread_of_the_byte_map():
+    """SIGMA_LN_R (tests/helpers.py): the standard deviation of
+    ln value(rint(u + 95.65)) - (u/8 + 5) ln 2 over the normal codes, and the
+    range of that log error (half a code plus the mantissa's linear
+    approximation of 2^x, about 7% either way)."""
+    from tests.helpers import SIGMA_LN_R
+    u = np.linspace(-56.0, 0.0, 4_000_001)
+    c = f8.expcast_codes(u)
+    assert c.min() >= 8                                      # all normal
+    lnr = np.log(f8.e4m3_values(c)) - (u / 8 + f8.P_SHIFT) * math.log(2)
+    assert abs(lnr.std() - SIGMA_LN_R) < 5e-4
+    assert np.abs(lnr).max() < 0.075
+    assert abs(lnr.mean()) < 0.01                            # beta centres it
+
+
+def test_plain_closed_forms():
+    scale = 1 / math.sqrt(128)
+    # Q = 0: every byte is 96 (value 2^5), so O is the mean of V-Smooth's
+    # reconstruction and LSE = ln n exactly
+    q, k, v = _qkv(1, 2, 130, 300, 15)
+    q.zero_()
+    o, lse = f8.attention_fp8_plain(_bits(q), _bits(k), _bits(v), scale)
+    _, _, vd = _dequantized(q, k, v)
+    for h in range(2):
+        assert np.allclose(o[0, :, h], vd[0, :, h].mean(axis=0), rtol=0, atol=1e-12)
+        assert np.allclose(lse[0, h], math.log(300), rtol=0, atol=1e-12)
+    # block-causal Q = 0: the mean over the allowed prefix, LSE = ln |A(i)|
+    o, lse = f8.attention_fp8_plain(_bits(q), _bits(k[:, :130]), _bits(v[:, :130]), scale, MASK_BLOCK_CAUSAL, 50)
+    _, _, vd = _dequantized(q, k[:, :130], v[:, :130])
+    for i in (0, 49, 50, 129):
+        n = min(130, (i // 50 + 1) * 50)
+        assert np.allclose(o[0, i, 1], vd[0, :n, 1].mean(axis=0), rtol=0, atol=1e-12)
+        assert lse[0, 1, i] == pytest.approx(math.log(n), abs=1e-12)
+    # constant V comes back exactly
+    q, k, v = _qkv(1, 1, 200, 333, 16)
+    v = torch.full_like(v, 0.625)
+    o, _ = f8.attention_fp8_plain(_bits(q), _bits(k), _bits(v), scale)
+    assert np.allclose(o, 0.625, rtol=1e-12)
+    # one dominant key selects its reconstructed value row; LSE is its logit
+    q, k, v = _qkv(1, 1, 4, 256, 17)
+    q = torch.zeros_like(q)
+    q[0, :, 0, 0] = 8.0
+    k = torch.zeros_like(k)
+    k[0, 200, 0, 0] = 8.0
+    o, lse = f8.attention_fp8_plain(_bits(q), _bits(k), _bits(v), 1.0)
+    _, _, vd = _dequantized(q, k, v)
+    for i in range(4):
+        assert np.allclose(o[0, i, 0], vd[0, 200, 0], rtol=0, atol=1e-9)
+        assert lse[0, 0, i] == pytest.approx(64.0, abs=0.05)
+
+
+def test_plain_statement_is_close_to_exact_softmax_on_the_same_operands():
+    """Only ExpCast separates the plain statement from exact attention on the
+    dequantised tensors: within the page's per-row total-variation scale."""
+    q, k, v = _qkv(1, 2, 600, 600, 18, scale_q=2.0)
+    scale = 1 / math.sqrt(128)
+    o8, l8 = f8.attention_fp8_plain(_bits(q), _bits(k), _bits(v), scale)
+    qd, kd, vd = _dequantized(q, k, v)
+    od, ld = _sdpa64(qd, kd, vd, scale, MASK_FULL, 0)
+    tv = golden()["row_tv_bound_percent"] / 100
+    assert _rel(o8, od) < tv
+    assert np.abs(l8 - ld).max() < tv
+
+
+@pytest.mark.parametrize("mask,chunk,sort_keys", [(MASK_FULL, 0, False), (MASK_FULL, 0, True),
+                                                  (MASK_BLOCK_CAUSAL, 300, False)])
+def test_tiled_schedule_stays_within_the_derived_bound_of_the_plain_statement(mask, chunk, sort_keys):
+    """The schedule the kernel uses (attention_fp8: 128-key tiles, lazily raised
+    reference on a grid) against the plain statement, under the bars the GPU
+    test applies to the kernel (tests/helpers.py); zeros, a 10% gain and
+    shuffled rows must fail those bars."""
+    from tests.helpers import check_expcast_parity
+    B, H, S = 1, 2, 1000
+    q, k, v = _qkv(B, H, S, S, 19, scale_q=1.5)
+    if sort_keys:
+        order = torch.argsort(k[0].float().sum(-1).mean(-1))   # every tile raises the reference
+        k, v = k[:, order], v[:, order]
+    scale = 1 / math.sqrt(128)
+    quant = (f8.quantize_qk(_bits(q)), f8.quantize_qk(_bits(k)), f8.vsmooth(_bits(v)))
+    o_t, l_t = f8.attention_fp8(None, None, None, scale, mask, chunk, quantized=quant)
+    o_p, l_p, s_o, s_l = f8.attention_fp8_plain(None, None, None, scale, mask, chunk, quantized=quant, spread=True)
+    flat = lambda a: np.concatenate([a[0, :, h] for h in range(H)])      # noqa: E731
+    flat_l = lambda a: np.concatenate([a[0, h] for h in range(H)])       # noqa: E731
+    groups = [np.arange(i * S, (i + 1) * S) for i in range(H)]
+    res = check_expcast_parity(flat(o_t), flat(o_p), flat_l(l_t), flat_l(l_p), flat(s_o), flat_l(s_l), groups)
+    assert res["ok"], res
+    assert res["rel_rms"] < 0.06
+    for bad in (np.zeros_like(o_t), 1.1 * o_t, o_t[:, np.random.default_rng(0).permutation(S)]):
+        assert not check_expcast_parity(flat(bad), flat(o_p), None, None, flat(s_o), None, groups)["ok"]

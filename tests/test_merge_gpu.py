@@ -70,3 +70,38 @@ def test_empty_partials():
     vb.vdit_attn_merge(a_o, a_l, empty_o, empty_l, B, H, S, D)
     torch.cuda.synchronize()
     assert torch.all(a_o == 0) and torch.all(torch.isneginf(a_l))
+
+
+def test_fp32_running_merge_over_eight_shards():
+    """vdit_attn_merge_f32: eight uneven K/V shards folded into an fp32 running
+    result that starts at (0, -inf); the last fold also writes the bf16 output,
+    which must be the running O rounded to nearest even."""
+    dev = torch.device("cuda:0")
+    B, H, Sq, D = 1, 3, 640, 128
+    shards = [300, 128, 457, 77, 512, 1, 260, 700]
+    q, k, v = wl.draw_qkv(B, H, Sq, sum(shards), D, seed=62, recipe="rms_qk")
+    qd = q.to(dev)
+    scale = 1 / math.sqrt(D)
+    o_acc = torch.zeros((B, Sq, H, D), dtype=torch.float32, device=dev)
+    lse_acc = torch.full((B, H, Sq), float("-inf"), dtype=torch.float32, device=dev)
+    o_out = torch.empty((B, Sq, H, D), dtype=torch.bfloat16, device=dev)
+    start = 0
+    for i, n in enumerate(shards):
+        kd = k[:, start:start + n].contiguous().to(dev)
+        vd = v[:, start:start + n].contiguous().to(dev)
+        o, lse = vb.attention(qd, kd, vd, scale, vb.VDIT_MASK_CROSS if n <= 512 else vb.VDIT_MASK_FULL)
+        vb.vdit_attn_merge_f32(o_acc, lse_acc, o, lse, o_out if i + 1 == len(shards) else None, B, H, Sq, D)
+        if i == 0:
+            torch.cuda.synchronize()
+            assert torch.equal(o_acc, o.float()) and torch.equal(lse_acc, lse)  # the first fold copies exactly
+        start += n
+    assert vb.vdit_get_device_status()[0] == vb.VDIT_OK
+    assert torch.equal(o_out, o_acc.to(torch.bfloat16))
+    o_r, l_r = oracle_attention(wl.bf16_bits(q), wl.bf16_bits(k), wl.bf16_bits(v), scale, vb.VDIT_MASK_CROSS)
+    o_g = o_out.float().cpu().numpy().astype(np.float64)
+    l_g = lse_acc.cpu().numpy().astype(np.float64)
+    og = np.concatenate([o_g[b, :, h] for b in range(B) for h in range(H)])
+    orr = np.concatenate([o_r[b, :, h] for b in range(B) for h in range(H)])
+    groups = [np.arange(i * Sq, (i + 1) * Sq) for i in range(B * H)]
+    res = check_parity(og, orr, l_g.reshape(-1), l_r.reshape(-1), groups, "fp32 merge, 8 shards")
+    assert res["ok"], res

@@ -39,6 +39,7 @@ EXPORTS = (
     "vdit_attn_fwd_ws",
     "vdit_attn_fwd_block_sparse",
     "vdit_attn_merge",
+    "vdit_attn_merge_f32",
     "vdit_attn_fwd_qknorm",
     "vdit_attn_qknorm_plan",
     "vdit_qk_rms_norm",
@@ -118,6 +119,8 @@ def lib() -> ctypes.CDLL:
             h.vdit_qk_rms_norm.argtypes = [vp, vp, vp, vp, vp, vp, c_float, c_int, c_int, c_int, c_int, c_int, vp]
             h.vdit_attn_merge.restype = c_int
             h.vdit_attn_merge.argtypes = [vp, vp, vp, vp, c_int, c_int, c_int, c_int, vp]
+            h.vdit_attn_merge_f32.restype = c_int
+            h.vdit_attn_merge_f32.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, vp]
             h.vdit_testing_attn_fwd.restype = c_int
             h.vdit_testing_attn_fwd.argtypes = fwd_args + [c_int, ctypes.c_ulonglong, vp]
             h.vdit_get_device_status.restype = c_int
@@ -360,6 +363,16 @@ def vdit_attn_merge(o_acc, lse_acc, o_part, lse_part, B, H, S, D, stream=None, c
                                _stream(stream))
     if check and st != VDIT_OK:
         raise VditError(st, "vdit_attn_merge")
+    return st
+
+
+def vdit_attn_merge_f32(o_acc, lse_acc, o_part, lse_part, o_out, B, H, S, D, stream=None, check=True) -> int:
+    """Fold (o_part, lse_part) into an fp32 running (o_acc, lse_acc); o_out (bf16, optional) also receives the
+    merged O rounded to bf16 (see include/vdit_attn.h)."""
+    st = lib().vdit_attn_merge_f32(_addr(o_acc), _addr(lse_acc), _addr(o_part), _addr(lse_part), _addr(o_out),
+                                   B, H, S, D, _stream(stream))
+    if check and st != VDIT_OK:
+        raise VditError(st, "vdit_attn_merge_f32")
     return st
 
 

@@ -485,6 +485,44 @@ vdit_status fp8_attention_impl(void* o, float* lse, const Shape& s, float scale,
                                                                                                   : VDIT_ERR_CUDA;
 }
 
+// ------------------------------------------------------------ LSE merge
+
+// Validates and queues one fold of (o_part, lse_part) into (o_acc, lse_acc);
+// AccT is the running O's storage (bf16 or fp32), o_out an optional bf16
+// copy of the merged O.
+template <typename AccT>
+vdit_status merge_impl(AccT* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out, int B,
+                       int H, int S, int D, cudaStream_t stream) {
+    if (B < 0 || H < 0 || S < 0 || D < 1) return VDIT_ERR_INVALID_ARG;
+    if (D != vdit::kHeadDim) return VDIT_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0 || S == 0) return VDIT_OK;
+    if (o_acc == nullptr || lse_acc == nullptr || o_part == nullptr || lse_part == nullptr)
+        return VDIT_ERR_INVALID_ARG;
+    if (!aligned16(o_acc) || !aligned16(o_part) || !aligned16(lse_acc) || !aligned16(lse_part) || !aligned16(o_out))
+        return VDIT_ERR_MISALIGNED;
+    const long long rows = (long long)B * S * H;
+    const long long warps = (long long)B * H * ((S + vdit::kMergeRowsPerWarp - 1) / vdit::kMergeRowsPerWarp);
+    const long long blocks = (warps + vdit::kMergeWarpsPerBlock - 1) / vdit::kMergeWarpsPerBlock;
+    if (blocks > 0x7fffffffLL) return VDIT_ERR_INVALID_ARG;
+    const size_t acc_bytes = size_t(rows) * size_t(D) * sizeof(AccT);
+    const size_t o_bytes = size_t(rows) * size_t(D) * 2, l_bytes = size_t(rows) * 4;
+    if (overlaps(o_acc, acc_bytes, o_part, o_bytes) || overlaps(lse_acc, l_bytes, lse_part, l_bytes) ||
+        overlaps(o_acc, acc_bytes, lse_acc, l_bytes) || overlaps(o_acc, acc_bytes, lse_part, l_bytes) ||
+        overlaps(lse_acc, l_bytes, o_part, o_bytes))
+        return VDIT_ERR_INVALID_ARG;
+    if (o_out != nullptr &&
+        (overlaps(o_out, o_bytes, o_acc, acc_bytes) || overlaps(o_out, o_bytes, o_part, o_bytes) ||
+         overlaps(o_out, o_bytes, lse_acc, l_bytes) || overlaps(o_out, o_bytes, lse_part, l_bytes)))
+        return VDIT_ERR_INVALID_ARG;
+    int dev = 0;
+    const vdit_status st = ensure_device(&dev);
+    if (st != VDIT_OK) return st;
+    vdit::attn_merge_kernel<AccT><<<unsigned(blocks), vdit::kMergeWarpsPerBlock * 32, 0, stream>>>(
+        o_acc, lse_acc, static_cast<const __nv_bfloat16*>(o_part), lse_part, static_cast<__nv_bfloat16*>(o_out), B,
+        H, S);
+    return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
+}
+
 }  // namespace
 
 // ------------------------------------------------------------ fixed scratch, no allocation
@@ -499,17 +537,31 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[VDIT_NOALLOC_SC
 namespace {
 
 struct NoAllocScratch {
-    std::once_flag once;
-    cudaError_t err = cudaErrorUnknown;
-    void* ptr = nullptr;
+    std::mutex mu;
+    void* ptr = nullptr;  // device address of g_noalloc_scratch on this device, once a lookup succeeded
 };
 NoAllocScratch g_noalloc[kMaxDevices];
 
-// Called with `dev` current (the entry point runs it for the current device).
-void resolve_noalloc_scratch(NoAllocScratch* st) {
-    void* p = nullptr;
-    st->err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    st->ptr = st->err == cudaSuccess ? p : nullptr;
+// The scratch's device address on `dev`, which must be the current device.
+// Only a successful lookup is cached, so a first call that failed (one made
+// during a stream capture, say) is retried by the next call instead of
+// failing for the rest of the process.  A cudaDeviceReset unloads the module
+// that holds the array, after which the cached address is stale: like the
+// per-device kernel attributes this library sets once, it assumes the device
+// is not reset while the library is in use.
+vdit_status noalloc_scratch(int dev, void** out) {
+    NoAllocScratch* sc = &g_noalloc[dev];
+    std::lock_guard<std::mutex> lock(sc->mu);
+    if (sc->ptr == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+            (void)cudaGetLastError();  // leave no error behind for the next launch check
+            return VDIT_ERR_CUDA;
+        }
+        sc->ptr = p;
+    }
+    *out = sc->ptr;
+    return VDIT_OK;
 }
 
 }  // namespace
@@ -649,23 +701,27 @@ vdit_status vdit_attn_fwd_qknorm_noalloc(const void* q, const void* k, const voi
                                          int H, int Sq, int Skv, int D, float scale, int mask_kind,
                                          int chunk_tokens, void* stream) {
     try {
+        // the argument checks of vdit_attn_fwd_qknorm, in its order, so that
+        // the two entry points accept and reject the same calls
         if (mask_kind == VDIT_MASK_BLOCK_SPARSE) return VDIT_ERR_INVALID_ARG;
         const Shape s{B, H, Sq, Skv, D, mask_kind, chunk_tokens};
-        const vdit_status st = check_shape(s, true, scale);
+        vdit_status st = check_shape(s, true, scale);
         if (st != VDIT_OK) return st;
+        if (!(std::isfinite(eps) && eps > 0.0f)) return VDIT_ERR_INVALID_ARG;
+        if (!aligned16(q_norm_weight) || !aligned16(k_norm_weight)) return VDIT_ERR_MISALIGNED;
         if (B == 0 || H == 0 || Sq == 0) return VDIT_OK;
         if (qknorm_workspace_bytes(B, H, Sq, Skv, D) > size_t(VDIT_NOALLOC_SCRATCH_BYTES))
             return VDIT_ERR_WORKSPACE;  // the shape does not fit the fixed scratch
         int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess) return VDIT_ERR_CUDA;
-        if (dev < 0 || dev >= kMaxDevices) return VDIT_ERR_UNSUPPORTED;
-        NoAllocScratch* sc = &g_noalloc[dev];
-        std::call_once(sc->once, resolve_noalloc_scratch, sc);
-        if (sc->err != cudaSuccess || sc->ptr == nullptr) return VDIT_ERR_CUDA;
+        st = ensure_device(&dev);  // an unsupported GPU reports VDIT_ERR_UNSUPPORTED before any lookup
+        if (st != VDIT_OK) return st;
+        void* scratch = nullptr;
+        st = noalloc_scratch(dev, &scratch);
+        if (st != VDIT_OK) return st;
         // Nothing in the scratch has to start at zero: the norm writes all of
         // the normalised Q and K before the attention reads them.
         return vdit_attn_fwd_qknorm(q, k, v, o, lse, q_norm_weight, k_norm_weight, eps, B, H, Sq, Skv, D, scale,
-                                    mask_kind, chunk_tokens, sc->ptr, size_t(VDIT_NOALLOC_SCRATCH_BYTES), stream);
+                                    mask_kind, chunk_tokens, scratch, size_t(VDIT_NOALLOC_SCRATCH_BYTES), stream);
     } catch (...) {
         return VDIT_ERR_CUDA;
     }
@@ -859,30 +915,18 @@ vdit_status vdit_testing_attn_fwd(const void* q, const void* k, const void* v, v
 vdit_status vdit_attn_merge(void* o_acc, float* lse_acc, const void* o_part, const float* lse_part, int B, int H,
                             int S, int D, void* stream) {
     try {
-        if (B < 0 || H < 0 || S < 0 || D < 1) return VDIT_ERR_INVALID_ARG;
-        if (D != vdit::kHeadDim) return VDIT_ERR_UNSUPPORTED;
-        if (B == 0 || H == 0 || S == 0) return VDIT_OK;
-        if (o_acc == nullptr || lse_acc == nullptr || o_part == nullptr || lse_part == nullptr)
-            return VDIT_ERR_INVALID_ARG;
-        if (!aligned16(o_acc) || !aligned16(o_part) || !aligned16(lse_acc) || !aligned16(lse_part))
-            return VDIT_ERR_MISALIGNED;
-        const long long rows = (long long)B * S * H;
-        const long long warps = (long long)B * H * ((S + vdit::kMergeRowsPerWarp - 1) / vdit::kMergeRowsPerWarp);
-        const long long blocks = (warps + vdit::kMergeWarpsPerBlock - 1) / vdit::kMergeWarpsPerBlock;
-        if (blocks > 0x7fffffffLL) return VDIT_ERR_INVALID_ARG;
-        const size_t o_bytes = size_t(rows) * size_t(D) * 2, l_bytes = size_t(rows) * 4;
-        if (overlaps(o_acc, o_bytes, o_part, o_bytes) || overlaps(lse_acc, l_bytes, lse_part, l_bytes) ||
-            overlaps(o_acc, o_bytes, lse_acc, l_bytes) || overlaps(o_acc, o_bytes, lse_part, l_bytes) ||
-            overlaps(lse_acc, l_bytes, o_part, o_bytes))
-            return VDIT_ERR_INVALID_ARG;
-        int dev = 0;
-        const vdit_status st = ensure_device(&dev);
-        if (st != VDIT_OK) return st;
-        vdit::attn_merge_kernel<<<unsigned(blocks), vdit::kMergeWarpsPerBlock * 32, 0,
-                                  static_cast<cudaStream_t>(stream)>>>(
-            static_cast<__nv_bfloat16*>(o_acc), lse_acc, static_cast<const __nv_bfloat16*>(o_part), lse_part, B, H,
-            S);
-        return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
+        return merge_impl(static_cast<__nv_bfloat16*>(o_acc), lse_acc, o_part, lse_part, nullptr, B, H, S, D,
+                          static_cast<cudaStream_t>(stream));
+    } catch (...) {
+        return VDIT_ERR_CUDA;
+    }
+}
+
+vdit_status vdit_attn_merge_f32(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                                void* o_out, int B, int H, int S, int D, void* stream) {
+    try {
+        return merge_impl(o_acc, lse_acc, o_part, lse_part, static_cast<__nv_bfloat16*>(o_out), B, H, S, D,
+                          static_cast<cudaStream_t>(stream));
     } catch (...) {
         return VDIT_ERR_CUDA;
     }
