@@ -8,10 +8,15 @@ sequences, it adds two scale-aware bars that an all-zero or shuffled O cannot
 pass: rms(err) / rms(O_ref) <= 1e-2 per (b, h), and cosine(O, O_ref) >= 0.9999.
 (bf16 rounding of O alone contributes about 2^-9 / sqrt(3) ~ 1e-3 to the first.)
 
-It also measures max|err| / rms(O_ref) per (b, h), in two forms: against the
+It also measures max|err| / rms(O_ref) per (b, h), in three forms: against the
 oracle rounded to bf16 (where a one-ulp rounding disagreement at the largest
-|O| of a head counts in full) and against the unrounded fp64 oracle (the
-kernel's own error, its final bf16 rounding included).  With the environment
+|O| of a head counts in full), against the unrounded fp64 oracle (the
+kernel's own error, its final bf16 rounding included), and the excess over
+that rounding: max(|O - O_ref| - 2^-8 max(|O|, |O_ref|), 0) / rms(O_ref), since
+rounding a value to bf16 moves it by at most 2^-8 of itself -- the last both
+per head and per head dim (each dim against its own rms, so that a channel
+whose values are several times larger, like the value-outlier channels of the
+480p workload, is held to the same relative bar as the others).  With the environment
 variable VDIT_PARITY_REPORT set to a file path, every call appends its
 measured figures to that file as one JSON line.
 """
@@ -62,16 +67,24 @@ def check_parity(o_gpu, o_ref, lse_gpu, lse_ref, group_rows=None, label=""):
            "max_over_bound": float((err / bound).max())}
     groups = group_rows if group_rows is not None else [np.arange(o_gpu.shape[0])]
     err_exact = np.abs(o_gpu - np.asarray(o_ref, dtype=np.float64))
-    worst_rel = worst_max_rms = worst_max_rms_exact = 0.0
+    excess = np.maximum(err_exact - 2.0 ** -8 * np.maximum(np.abs(o_gpu), np.abs(np.asarray(o_ref, np.float64))),
+                        0.0)
+    worst_rel = worst_max_rms = worst_max_rms_exact = worst_excess = worst_excess_ch = 0.0
     for g in groups:
         rms = max(float(np.sqrt(np.mean(o_ref[g] ** 2))), 1e-30)
         rms_err = float(np.sqrt(np.mean(err[g] ** 2)))
         worst_rel = max(worst_rel, rms_err / rms)
         worst_max_rms = max(worst_max_rms, float(err[g].max()) / rms)
         worst_max_rms_exact = max(worst_max_rms_exact, float(err_exact[g].max()) / rms)
+        worst_excess = max(worst_excess, float(excess[g].max()) / rms)
+        # per channel: each head dim against its own rms over the group's rows
+        rms_ch = np.maximum(np.sqrt(np.mean(np.asarray(o_ref[g], np.float64) ** 2, axis=0)), 1e-30)
+        worst_excess_ch = max(worst_excess_ch, float((excess[g] / rms_ch).max()))
     res["rel_rms_err"] = worst_rel
     res["max_over_rms"] = worst_max_rms
     res["max_over_rms_exact"] = worst_max_rms_exact
+    res["max_excess_over_rms"] = worst_excess
+    res["max_excess_over_channel_rms"] = worst_excess_ch
     a, b = o_gpu.ravel(), np.asarray(o_ref, dtype=np.float64).ravel()
     res["cosine"] = float(a @ b / max(np.linalg.norm(a) * np.linalg.norm(b), 1e-300))
     if lse_gpu is not None:
@@ -113,8 +126,10 @@ def check_parity(o_gpu, o_ref, lse_gpu, lse_ref, group_rows=None, label=""):
 # head dim, computed by the plain oracle.  Likewise LSE_k - LSE_p = ln sum_j
 # w_j e^lambda_j, within sigma_lambda sqrt(sum_j w_j^2) of the mean of lambda,
 # which is zero over a uniform spread of u.  The bars:
-#   per element  |O_k - O_p| <= 8 sigma_lambda spread + 2^-8 |O_p| + 1e-6
-#                (8 standard deviations; 2^-8 |O|: the kernel's bf16 rounding)
+#   per element  |O_k - O_p| <= 8 sigma_lambda spread + 2^-7 |O_p| + 1e-6
+#                (8 standard deviations; 2^-7 |O|: the kernel's bf16 output,
+#                one ulp, since its fp32 value may sit on the far side of a
+#                rounding boundary from the plain value)
 #   per (b, h)   rms(O_k - O_p) <= sigma_lambda rms(spread) + 2^-9 rms(O_p)
 #   per row      |LSE_k - LSE_p| <= 8 sigma_lambda sqrt(sum_j w_j^2) + 1e-4
 SIGMA_LN_R = 0.0313
@@ -128,7 +143,7 @@ def check_expcast_parity(o_gpu, o_plain, lse_gpu, lse_plain, spread_o, spread_l,
     o_gpu = np.asarray(o_gpu, dtype=np.float64)
     o_plain = np.asarray(o_plain, dtype=np.float64)
     d = np.abs(o_gpu - o_plain)
-    bound = EXPCAST_K * SIGMA_LAMBDA * spread_o + 2.0 ** -8 * np.abs(o_plain) + 1e-6
+    bound = EXPCAST_K * SIGMA_LAMBDA * spread_o + 2.0 ** -7 * np.abs(o_plain) + 1e-6
     res = {"label": label, "max_over_bound": float((d / bound).max()),
            "max_d_over_spread": float((d / np.maximum(spread_o, 1e-30)).max())}
     groups = group_rows if group_rows is not None else [np.arange(o_gpu.shape[0])]
