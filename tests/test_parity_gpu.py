@@ -193,15 +193,17 @@ def test_bitwise_deterministic():
         assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
-def test_writes_stay_inside_the_output_buffers():
+@pytest.mark.parametrize("mask,Skv", [(FULL, 300), (CROSS, 77)])
+def test_writes_stay_inside_the_output_buffers(mask, Skv):
+    # the cross kernel stores O with TMA boxes of 32 rows: Sq = 300 ends inside one
     dev = torch.device("cuda:0")
     B, H, Sq, D = 1, 2, 300, 128
-    q, k, v = (t.to(dev) for t in wl.draw_qkv(B, H, Sq, Sq, D, seed=16))
+    q, k, v = (t.to(dev) for t in wl.draw_qkv(B, H, Sq, Skv, D, seed=16))
     n_o, n_l, guard = B * Sq * H * D, B * H * Sq, 4096
     o_buf = torch.full((n_o + guard,), 7.0, dtype=torch.bfloat16, device=dev)
     l_buf = torch.full((n_l + guard,), 7.0, dtype=torch.float32, device=dev)
-    vb.vdit_attn_fwd(q, k, v, o_buf.data_ptr(), l_buf.data_ptr(), B, H, Sq, Sq, D, 1 / math.sqrt(D),
-                     FULL, 0)
+    vb.vdit_attn_fwd(q, k, v, o_buf.data_ptr(), l_buf.data_ptr(), B, H, Sq, Skv, D, 1 / math.sqrt(D),
+                     mask, 0)
     torch.cuda.synchronize()
     assert torch.all(o_buf[n_o:] == 7.0) and torch.all(l_buf[n_l:] == 7.0)
     assert torch.isfinite(o_buf[:n_o].float()).all() and torch.isfinite(l_buf[:n_l]).all()

@@ -60,9 +60,14 @@ struct __align__(8) CrossBarriers {
     int abort;
 };
 
+constexpr int kCrossStageRows = 32;   // epilogue: one warp's rows
+constexpr int kCrossStageCols = 32;   // head dims per staged chunk (64 bytes of a bf16 row)
+constexpr int kCrossStageBytes = kCrossStageRows * kCrossStageCols * 2;  // 2 KB per softmax warp
+
 constexpr int kCrossSmemQ = 0;
 constexpr int kCrossSmemKV = kTileBytes;
-constexpr int kCrossSmemBar = kCrossSmemKV + 2 * kTileBytes;
+constexpr int kCrossSmemStage = kCrossSmemKV + 2 * kTileBytes;  // 4 x 2 KB: the epilogue's store staging
+constexpr int kCrossSmemBar = kCrossSmemStage + 4 * kCrossStageBytes;
 constexpr int kCrossSmemBytes = kCrossSmemBar + ((int(sizeof(CrossBarriers)) + 15) / 16) * 16 + 1024;  // + alignment
 
 // Item i is query tile i % n_qb of (batch, head) i / n_qb: the CTAs running at
@@ -74,9 +79,12 @@ __device__ __forceinline__ void cross_item(const FwdParams& p, long long item, i
     b = static_cast<int>(bh / p.H);
 }
 
+// tm_o: O as the same 4-D tensor as Q, with 32-dim x 32-row boxes and no
+// swizzle: the epilogue's TMA store unit.
 __global__ void __launch_bounds__(kCrossThreads, 2)
     attn_cross_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                            const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                            const FwdParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw_base + 1023u) & ~1023u) - raw_base);
@@ -106,6 +114,7 @@ __global__ void __launch_bounds__(kCrossThreads, 2)
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_o);
     }
     if (warp == kCrossMmaWarp) {
         tmem_alloc(smem_addr(&bars->tmem_base), kCrossTmemCols);
@@ -323,10 +332,16 @@ __global__ void __launch_bounds__(kCrossThreads, 2)
                 int b, h, q0;
                 cross_item(p, item, b, h, q0);
                 const int row = q0 + row_in_tile;
+                const int warp_row0 = q0 + warp * kCrossStageRows;  // first row of this warp's TMA boxes
                 const float inv_l = 1.0f / l;  // l >= 1: the row's maximum key contributes 2^0
-                __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.Sq + row) * p.H + h) * kHeadDim;
+                // O leaves through shared memory, 32 head dims at a time: each
+                // thread writes its row's 64 bytes into the warp's 2 KB staging
+                // box, and one TMA store moves the 32 x 32 box to global memory,
+                // instead of 32 rows of 16-byte pieces per store instruction.
+                uint8_t* stage = smem + kCrossSmemStage + warp * kCrossStageBytes;
+                const uint32_t stage_addr = smem_addr(stage);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < kHeadDim / kCrossStageCols; ++c) {
                     uint32_t o[32];
                     tmem_ld32(tO + uint32_t(c) * 32u, o);
                     tmem_ld_wait(o);
@@ -334,11 +349,17 @@ __global__ void __launch_bounds__(kCrossThreads, 2)
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
                         pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-                    if (row < p.Sq) {
-                        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+                    // the previous box's store has read the staging buffer
+                    if (lane == 0) bulk_wait_read_all();
+                    __syncwarp();
+                    uint4* dst = reinterpret_cast<uint4*>(stage + lane * (kCrossStageCols * 2));
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && warp_row0 < p.Sq) {
+                        tma_store_4d(&tm_o, stage_addr, c * kCrossStageCols, h, warp_row0, b);
+                        bulk_commit_group();
                     }
                 }
                 if (p.lse != nullptr && row < p.Sq)
@@ -349,6 +370,7 @@ __global__ void __launch_bounds__(kCrossThreads, 2)
     }
 
     // ------------------------------------------------ teardown
+    if (warp < 4 && lane == 0) bulk_wait_all();  // the epilogue's stores are complete
     tc_fence_before_sync();
     __syncthreads();
     if (warp == kCrossMmaWarp) {

@@ -72,7 +72,8 @@ constexpr int kMaskCross = 2;
 constexpr int kMaskBlockSparse = 3;
 constexpr int kSparseBlock = 128;        // block-mask granularity = the 128-row/128-key tiles
 constexpr int kMaxSparseKvBlocks = 2048; // key blocks a block-sparse call may have (Skv <= 262,144)
-constexpr uint16_t kListKvMask = 0x3FFF; // list entry: key block | allowed for tile 0 << 14 | tile 1 << 15
+constexpr int kMaxSparseEntries = 2 * kMaxSparseKvBlocks;  // both query tiles' key lists, interleaved
+constexpr uint16_t kListKvMask = 0x3FFF; // list entry: key block | owner query tile << 14
 constexpr int kListWarp = 10;
 
 // Device status word codes (OR-ed together).
@@ -98,6 +99,8 @@ constexpr int kSmemKV = kQTiles * kTileBytes;
 constexpr int kSmemBar = kSmemKV + kStages * kTileBytes;
 constexpr int kSmemList = kSmemBar + ((int(sizeof(Barriers)) + 15) / 16) * 16;  // block-sparse tile list
 constexpr int kSmemBytes = kSmemList + kMaxSparseKvBlocks * 2 + 16 + 1024;     // + alignment slack
+// the block-sparse instantiation holds both tiles' key lists (twice the room)
+constexpr int kSmemBytesSparse = kSmemList + kMaxSparseEntries * 2 + 16 + 1024;
 
 struct FwdParams {
     int B, H, Sq, Skv;
@@ -221,10 +224,21 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&s)[32], uint64_t scal
 
 // ---------------------------------------------------------------- kernel
 
-// kSparse: the block-sparse instantiation, whose query tiles each take part
-// only in the key tiles their own mask rows allow.  The dense, block-causal
-// and cross instantiation keeps the plain issue order, in which both tiles
-// take part in every key tile.
+// Position in the block-sparse stream of entry k of query tile t's key list,
+// when tile 0's list has n0 entries and tile 1's n1: the lists alternate
+// (0, 1, 0, 1, ...) while both last, then the longer one's rest follows.
+__device__ __forceinline__ int sparse_pos(int k, int t, int n0, int n1) {
+    const int both = min(n0, n1);
+    return k < both ? 2 * k + t : 2 * both + (k - both);
+}
+
+// kSparse: the block-sparse instantiation.  Each query tile walks only the
+// key blocks its own mask row allows; the two tiles' lists are interleaved
+// into one stream of (key block, owner tile) entries, which the producer
+// loads in order, so the tiles take turns with the tensor core and MUFU as
+// in the dense schedule.  A key block both tiles need appears once for each.
+// The dense, block-causal and cross instantiation keeps the plain issue
+// order, in which both tiles take part in every key tile.
 template <bool kSparse>
 __global__ void __launch_bounds__(kNumThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -267,25 +281,37 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         tmem_relinquish();
     }
     uint16_t* kv_list = reinterpret_cast<uint16_t*>(smem + kSmemList);
-    int* kv_list_len = reinterpret_cast<int*>(smem + kSmemList + kMaxSparseKvBlocks * 2);
+    int* kv_list_len = reinterpret_cast<int*>(smem + kSmemList + kMaxSparseEntries * 2);  // total, n0, n1 (sparse)
     if (kSparse && warp == kListWarp) {
-        // Compact the key blocks either query tile of this CTA attends to,
-        // in ascending order, each tagged with which of the two tiles may use it.
+        // Each query tile's allowed key blocks in ascending order, interleaved
+        // into one stream (sparse_pos), each entry tagged with its owner tile.
         const int qb0 = q0 / kSparseBlock;
         const uint8_t* row0 = p.block_mask + ((static_cast<size_t>(b) * p.H + h) * p.n_qb + qb0) * p.n_kvb;
         const bool has_row1 = qb0 + 1 < p.n_qb;
-        int count = 0;
+        const uint32_t below = (1u << lane) - 1u;
+        int n0 = 0, n1 = 0;
+        for (int base = 0; base < p.n_kvb; base += 32) {
+            const int kv = base + lane;
+            n0 += __popc(__ballot_sync(0xffffffffu, kv < p.n_kvb && row0[kv] != 0));
+            n1 += __popc(__ballot_sync(0xffffffffu, has_row1 && kv < p.n_kvb && row0[p.n_kvb + kv] != 0));
+        }
+        int c0 = 0, c1 = 0;
         for (int base = 0; base < p.n_kvb; base += 32) {
             const int kv = base + lane;
             const bool a0 = kv < p.n_kvb && row0[kv] != 0;
             const bool a1 = has_row1 && kv < p.n_kvb && row0[p.n_kvb + kv] != 0;
-            const uint32_t ballot = __ballot_sync(0xffffffffu, a0 || a1);
-            if (a0 || a1)
-                kv_list[count + __popc(ballot & ((1u << lane) - 1u))] =
-                    uint16_t(kv | (a0 ? 1 << 14 : 0) | (a1 ? 1 << 15 : 0));
-            count += __popc(ballot);
+            const uint32_t b0 = __ballot_sync(0xffffffffu, a0);
+            const uint32_t b1 = __ballot_sync(0xffffffffu, a1);
+            if (a0) kv_list[sparse_pos(c0 + __popc(b0 & below), 0, n0, n1)] = uint16_t(kv);
+            if (a1) kv_list[sparse_pos(c1 + __popc(b1 & below), 1, n0, n1)] = uint16_t(kv | (1 << 14));
+            c0 += __popc(b0);
+            c1 += __popc(b1);
         }
-        if (lane == 0) *kv_list_len = count;
+        if (lane == 0) {
+            kv_list_len[0] = n0 + n1;
+            kv_list_len[1] = n0;
+            kv_list_len[2] = n1;
+        }
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -391,70 +417,63 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 }
             }
             } else {
-            // A query tile takes part in key tile e unless a block-sparse entry
-            // leaves it out; its S and P V are then skipped, and its barrier
-            // phases count only the key tiles it takes part in.
-            auto part = [&](int e, int t) -> bool { return !sparse || ((kv_list[e] >> (14 + t)) & 1u); };
-            int last[2] = {n_kv - 1, n_kv - 1};  // each tile's last key tile (-1: none)
-            if (sparse) {
-                last[0] = last[1] = -1;
-                for (int e = n_kv - 1; e >= 0 && (last[0] < 0 || last[1] < 0); --e) {
-                    if (last[0] < 0 && part(e, 0)) last[0] = e;
-                    if (last[1] < 0 && part(e, 1)) last[1] = e;
-                }
-            }
-            int done[2] = {0, 0};  // P V products issued per tile
-            // prologue: the scores of the tiles that take part in key tile 0
-            if (ok) ok = bounded_wait(smem_addr(&bars->kv_full[0]), 0, abort_flag, p.timeout_ns, kSiteMma);
-            if (ok) {
+            // Block-sparse: stream entry e belongs to one query tile.  After
+            // that tile's P V on e comes its S on its next entry (two entries
+            // on while both lists last, then the next one), so the two tiles
+            // keep taking turns.  Barrier phases count each tile's own entries.
+            auto owner = [&](int e) -> int { return (kv_list[e] >> 14) & 1; };
+            auto next_own = [&](int e) -> int {  // the owner's next entry after e, or -1
+                const int t = owner(e);
+                for (int f = e + 1; f < n_kv; ++f)
+                    if (owner(f) == t) return f;
+                return -1;
+            };
+            int done0 = 0, done1 = 0;  // P V products issued per tile (scalars: no local-memory array)
+            // prologue: the scores of each tile's first entry (entries 0 and 1
+            // while both tiles have entries)
+            for (int e = 0; ok && e < 2 && e < n_kv; ++e) {
+                if (e == 1 && owner(1) == owner(0)) break;
+                ok = bounded_wait(smem_addr(&bars->kv_full[(2 * e) % kStages]), 0, abort_flag, p.timeout_ns, kSiteMma);
+                if (!ok) break;
                 tc_fence_after_sync();
-                for (int t = 0; t < kQTiles; ++t) {
-                    if (!part(0, t)) continue;
-                    issue_qk(tS[t], q_desc[t], k_desc0);
-                    umma_commit(smem_addr(&bars->s_full[t]));
-                }
-                umma_commit(smem_addr(&bars->kv_empty[0]));
+                const int t = owner(e);
+                issue_qk(t ? tS[1] : tS[0], t ? q_desc[1] : q_desc[0], k_desc0 + uint64_t((2 * e) % kStages) * kSlotStep);
+                umma_commit(smem_addr(&bars->s_full[t]));
+                umma_commit(smem_addr(&bars->kv_empty[(2 * e) % kStages]));
             }
-            // steady state, per key tile j (each step only for the tiles that take part):
-            //   PV0(j) [two halves]  S0(j+1)  PV1(j) [two halves]  S1(j+1)
-            for (int j = 0; ok && j < n_kv; ++j) {
-                const int uv = 2 * j + 1;
+            for (int e = 0; ok && e < n_kv; ++e) {
+                const int t = owner(e);
+                const int uv = 2 * e + 1;
                 const int v_slot = uv % kStages;
-                const int uk = 2 * (j + 1);
-                const int k_slot = uk % kStages;
-                const bool more = (j + 1) < n_kv;
-                bool k_ready = false;
                 ok = bounded_wait(smem_addr(&bars->kv_full[v_slot]), uint32_t(uv / kStages) & 1u, abort_flag,
                                   p.timeout_ns, kSiteMma);
-                for (int t = 0; ok && t < kQTiles; ++t) {
-                    if (part(j, t)) {
-                        const uint32_t ph = uint32_t(done[t]) & 1u;
-                        for (int hf = 0; ok && hf < 2; ++hf) {
-                            ok = bounded_wait(smem_addr(&bars->p_full[t][hf]), ph, abort_flag, p.timeout_ns,
-                                              kSiteMma);
-                            if (ok) {
-                                tc_fence_after_sync();
-                                issue_pv_half(tO[t], tS[t], v_desc0 + uint64_t(v_slot) * kSlotStep, hf, done[t] > 0);
-                            }
-                        }
-                        if (!ok) break;
-                        ++done[t];
-                        if (j == last[t]) umma_commit(smem_addr(&bars->o_full[t]));
-                    }
-                    if (t == 1) umma_commit(smem_addr(&bars->kv_empty[v_slot]));
-                    if (more && part(j + 1, t)) {
-                        if (!k_ready) {
-                            ok = bounded_wait(smem_addr(&bars->kv_full[k_slot]), uint32_t(uk / kStages) & 1u,
-                                              abort_flag, p.timeout_ns, kSiteMma);
-                            if (!ok) break;
-                            tc_fence_after_sync();
-                            k_ready = true;
-                        }
-                        issue_qk(tS[t], q_desc[t], k_desc0 + uint64_t(k_slot) * kSlotStep);
-                        umma_commit(smem_addr(&bars->s_full[t]));
+                const int done_t = t ? done1 : done0;
+                const uint32_t ph = uint32_t(done_t) & 1u;
+                for (int hf = 0; ok && hf < 2; ++hf) {
+                    ok = bounded_wait(smem_addr(&bars->p_full[t][hf]), ph, abort_flag, p.timeout_ns, kSiteMma);
+                    if (ok) {
+                        tc_fence_after_sync();
+                        issue_pv_half(t ? tO[1] : tO[0], t ? tS[1] : tS[0], v_desc0 + uint64_t(v_slot) * kSlotStep, hf,
+                                      done_t > 0);
                     }
                 }
-                if (ok && more) umma_commit(smem_addr(&bars->kv_empty[k_slot]));  // after every S of K_(j+1)
+                if (!ok) break;
+                umma_commit(smem_addr(&bars->kv_empty[v_slot]));
+                if (t) ++done1; else ++done0;
+                const int f = next_own(e);
+                if (f < 0) {
+                    umma_commit(smem_addr(&bars->o_full[t]));
+                } else if (f > 1 || owner(1) == owner(0)) {  // entries 0 and 1 of two tiles had theirs in the prologue
+                    const int uk = 2 * f;
+                    const int k_slot = uk % kStages;
+                    ok = bounded_wait(smem_addr(&bars->kv_full[k_slot]), uint32_t(uk / kStages) & 1u, abort_flag,
+                                      p.timeout_ns, kSiteMma);
+                    if (!ok) break;
+                    tc_fence_after_sync();
+                    issue_qk(t ? tS[1] : tS[0], t ? q_desc[1] : q_desc[0], k_desc0 + uint64_t(k_slot) * kSlotStep);
+                    umma_commit(smem_addr(&bars->s_full[t]));
+                    umma_commit(smem_addr(&bars->kv_empty[k_slot]));
+                }
             }
             }
             if (!ok) {
@@ -490,10 +509,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         float l = 0.0f;       // running row sum at that reference
         bool ok = true;
 
-        int taken = 0;  // key tiles this query tile has taken part in
-        for (int j = 0; j < n_kv; ++j) {
-            if (kSparse && !((kv_list[j] >> (14 + t)) & 1u)) continue;  // this tile sits this key tile out
-            const int idx = kSparse ? taken : j;  // this tile's count of key tiles so far
+        // key tiles this query tile takes part in: all n_kv, or its own block-sparse entries
+        const int n_mine = kSparse ? kv_list_len[1 + t] : n_kv;
+        for (int j = 0; j < n_mine; ++j) {
+            const int idx = j;
             ok = warp_wait(s_full, uint32_t(idx) & 1u, abort_flag, p.timeout_ns, kSiteSoftmax);
             if (!ok) break;
             tc_fence_after_sync();
@@ -506,8 +525,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             // keys of this tile allowed for the row: [0, lim) of the tile
             int lim;
             if (sparse) {
-                const uint32_t e = kv_list[j];
-                lim = ((e >> (14 + t)) & 1u) ? p.Skv - int(e & kListKvMask) * kBlockN : 0;
+                const int e = sparse_pos(j, t, kv_list_len[1], kv_list_len[2]);
+                lim = p.Skv - int(kv_list[e] & kListKvMask) * kBlockN;
             } else {
                 lim = kv_lim - j * kBlockN;
             }
@@ -605,13 +624,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     part += __uint_as_float(uint32_t(lsum[q])) + __uint_as_float(uint32_t(lsum[q] >> 32));
                 l += part;
             }
-            if (kSparse) ++taken;
         }
 
         // With no key tile for this query tile (nothing it attends to in a
         // block-sparse mask) O stays 0 and LSE = -inf; nothing was issued for
         // it, so there is nothing to wait for.
-        const int n_mine = kSparse ? taken : n_kv;  // key tiles this query tile took part in
         if (ok && n_mine > 0) ok = warp_wait(smem_addr(&bars->o_full[t]), 0, abort_flag, p.timeout_ns, kSiteSoftmax);
         if (ok) {
             tc_fence_after_sync();

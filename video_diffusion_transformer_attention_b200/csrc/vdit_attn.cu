@@ -87,7 +87,7 @@ void init_device(int dev, DeviceState* st) {
     if (cudaFuncSetAttribute(vdit::attn_fwd_sm100_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              vdit::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(vdit::attn_fwd_sm100_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             vdit::kSmemBytes) != cudaSuccess ||
+                             vdit::kSmemBytesSparse) != cudaSuccess ||
         cudaFuncSetAttribute(vdit::attn_cross_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              vdit::kCrossSmemBytes) != cudaSuccess ||
         // all of the unified L1 / shared storage as shared memory: two CTAs fit
@@ -163,6 +163,22 @@ bool encode_bshd(CUtensorMap* map, const void* base, int B, int S, int H) {
     return r == CUDA_SUCCESS;
 }
 
+// The output O as a store target for the cross-attention epilogue: the same
+// 4-D view, boxes of 32 head dims x 32 tokens, no swizzle (a warp's rows, one
+// 64-byte piece each).  Rows past S are not written.
+bool encode_bshd_store(CUtensorMap* map, void* base, int B, int S, int H) {
+    PFN_cuTensorMapEncodeTiled_v12000 f = encode_fn();
+    if (f == nullptr) return false;
+    const cuuint64_t D = vdit::kHeadDim;
+    cuuint64_t dims[4] = {D, cuuint64_t(H), cuuint64_t(S), cuuint64_t(B)};
+    cuuint64_t strides[3] = {D * 2, cuuint64_t(H) * D * 2, cuuint64_t(S) * cuuint64_t(H) * D * 2};
+    cuuint32_t box[4] = {cuuint32_t(vdit::kCrossStageCols), 1, cuuint32_t(vdit::kCrossStageRows), 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return f(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 vdit_status launch(const void* q, const void* k, const void* v, void* o, float* lse, const uint8_t* block_mask,
                    const Shape& s, float scale, int debug_flags, unsigned long long timeout_ns, cudaStream_t stream,
                    bool after_norm) {
@@ -193,8 +209,11 @@ vdit_status launch(const void* q, const void* k, const void* v, void* o, float* 
         // Short key sequence: persistent, two CTAs per SM, one 128-row query tile per item.
         const long long items = static_cast<long long>(p.n_qb) * s.H * s.B;
         const dim3 grid(static_cast<unsigned>(items < ds->cross_grid ? items : ds->cross_grid));
+        CUtensorMap to;
+        if (!encode_bshd_store(&to, o, s.B, s.Sq, s.H)) return VDIT_ERR_CUDA;
         if (!after_norm) {
-            vdit::attn_cross_sm100_kernel<<<grid, vdit::kCrossThreads, vdit::kCrossSmemBytes, stream>>>(tq, tk, tv, p);
+            vdit::attn_cross_sm100_kernel<<<grid, vdit::kCrossThreads, vdit::kCrossSmemBytes, stream>>>(tq, tk, tv, to,
+                                                                                                      p);
             return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
         }
         cudaLaunchConfig_t cfg{};
@@ -207,13 +226,15 @@ vdit_status launch(const void* q, const void* k, const void* v, void* o, float* 
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, vdit::attn_cross_sm100_kernel, tq, tk, tv, p) == cudaSuccess ? VDIT_OK
-                                                                                                     : VDIT_ERR_CUDA;
+        return cudaLaunchKernelEx(&cfg, vdit::attn_cross_sm100_kernel, tq, tk, tv, to, p) == cudaSuccess
+                   ? VDIT_OK
+                   : VDIT_ERR_CUDA;
     }
     dim3 grid(grid_x(s.Sq), s.H, s.B);
     if (!after_norm) {
         if (s.mask_kind == VDIT_MASK_BLOCK_SPARSE)
-            vdit::attn_fwd_sm100_kernel<true><<<grid, vdit::kNumThreads, vdit::kSmemBytes, stream>>>(tq, tk, tv, p);
+            vdit::attn_fwd_sm100_kernel<true><<<grid, vdit::kNumThreads, vdit::kSmemBytesSparse, stream>>>(tq, tk, tv,
+                                                                                                         p);
         else
             vdit::attn_fwd_sm100_kernel<false><<<grid, vdit::kNumThreads, vdit::kSmemBytes, stream>>>(tq, tk, tv, p);
         return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
