@@ -13,10 +13,12 @@ oracle rounded to bf16 (where a one-ulp rounding disagreement at the largest
 |O| of a head counts in full), against the unrounded fp64 oracle (the
 kernel's own error, its final bf16 rounding included), and the excess over
 that rounding: max(|O - O_ref| - 2^-8 max(|O|, |O_ref|), 0) / rms(O_ref), since
-rounding a value to bf16 moves it by at most 2^-8 of itself -- the last both
-per head and per head dim (each dim against its own rms, so that a channel
-whose values are several times larger, like the value-outlier channels of the
-480p workload, is held to the same relative bar as the others).  With the environment
+rounding a value to bf16 moves it by at most 2^-8 of itself -- the last per
+head, and per head dim against max(that dim's rms, the head's rms): a channel
+whose values are several times larger than the rest (the value-outlier
+channels of the 480p workload) has a proportionally larger error, and a
+channel whose outputs barely vary over the rows (a tiny scale) has a tiny rms
+of its own.  That last figure is held to EXCESS_BAR.  With the environment
 variable VDIT_PARITY_REPORT set to a file path, every call appends its
 measured figures to that file as one JSON line.
 """
@@ -31,6 +33,13 @@ MEAN_ABS = 1e-3
 LSE_REL = 1e-3
 REL_RMS_ERR = 1e-2
 MIN_COSINE = 0.9999
+# max(|O - O_ref| - 2^-8 max(|O|, |O_ref|), 0), the error beyond one bf16
+# rounding of the output, over max(rms of the head dim, rms of the head) per
+# (b, h): SURVEY's 2e-2 on max|err| / rms, read as a bar on what the output
+# rounding does not explain.  For outputs that are one kernel's fp32 result
+# rounded once to bf16; results composed of several rounded outputs (merged
+# partials, other arithmetic) pass excess_bar=None.
+EXCESS_BAR = 2e-2
 
 
 def to_bf16_bits(x) -> np.ndarray:
@@ -50,7 +59,7 @@ def round_bf16(x) -> np.ndarray:
     return bits_to_float(to_bf16_bits(np.asarray(x, dtype=np.float64)))
 
 
-def check_parity(o_gpu, o_ref, lse_gpu, lse_ref, group_rows=None, label=""):
+def check_parity(o_gpu, o_ref, lse_gpu, lse_ref, group_rows=None, label="", excess_bar=EXCESS_BAR):
     """Compare one call's outputs; returns a dict of the measured errors.
 
     o_gpu: [n, D] float (bf16 values), o_ref: [n, D] float64 oracle values.
@@ -77,8 +86,8 @@ def check_parity(o_gpu, o_ref, lse_gpu, lse_ref, group_rows=None, label=""):
         worst_max_rms = max(worst_max_rms, float(err[g].max()) / rms)
         worst_max_rms_exact = max(worst_max_rms_exact, float(err_exact[g].max()) / rms)
         worst_excess = max(worst_excess, float(excess[g].max()) / rms)
-        # per channel: each head dim against its own rms over the group's rows
-        rms_ch = np.maximum(np.sqrt(np.mean(np.asarray(o_ref[g], np.float64) ** 2, axis=0)), 1e-30)
+        # per head dim, against max(its own rms over the group's rows, the head's rms)
+        rms_ch = np.maximum(np.sqrt(np.mean(np.asarray(o_ref[g], np.float64) ** 2, axis=0)), rms)
         worst_excess_ch = max(worst_excess_ch, float((excess[g] / rms_ch).max()))
     res["rel_rms_err"] = worst_rel
     res["max_over_rms"] = worst_max_rms
@@ -95,7 +104,8 @@ def check_parity(o_gpu, o_ref, lse_gpu, lse_ref, group_rows=None, label=""):
         res["lse_rel"] = float(np.max(np.abs(lg - lr) / np.maximum(np.abs(lr), 1.0)))
     ok = (res["max_over_bound"] <= 1.0 and res["mean_abs"] <= MEAN_ABS
           and res["rel_rms_err"] <= REL_RMS_ERR and res["cosine"] >= MIN_COSINE
-          and (lse_gpu is None or res["lse_rel"] <= LSE_REL))
+          and (lse_gpu is None or res["lse_rel"] <= LSE_REL)
+          and (excess_bar is None or worst_excess_ch <= excess_bar))
     res["ok"] = bool(ok)
     res["label"] = label
     report = os.environ.get("VDIT_PARITY_REPORT")

@@ -112,7 +112,8 @@ def test_ring_attention_with_the_cuda_kernels(world, case):
         lg = np.concatenate([lse[b, h] for b in range(B) for h in range(H)])
         lr = np.concatenate([l_r[b, h, rank * s:(rank + 1) * s] for b in range(B) for h in range(H)])
         groups = [np.arange(i * s, (i + 1) * s) for i in range(B * H)]
-        res = check_parity(og, orr, lg, lr, groups, f"ring N={world} rank {rank}")
+        res = check_parity(og, orr, lg, lr, groups, f"ring N={world} rank {rank}",
+                           excess_bar=None)  # N partial outputs, each rounded to bf16, merged
         assert res["ok"], res
 
 

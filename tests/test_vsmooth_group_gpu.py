@@ -162,5 +162,6 @@ def test_grouping_shrinks_the_v_quantisation_error_and_keeps_attention_parity():
     og = np.concatenate([o_grp.float().cpu().numpy()[0, :, h] for h in range(H)]).astype(np.float64)
     orr = np.concatenate([o_r[0, :, h] for h in range(H)])
     lg = lse_grp.cpu().numpy().reshape(-1).astype(np.float64)
-    res = check_parity(og, orr, lg, l_r.reshape(-1), [np.arange(i * S, (i + 1) * S) for i in range(H)], "grouped")
+    res = check_parity(og, orr, lg, l_r.reshape(-1), [np.arange(i * S, (i + 1) * S) for i in range(H)], "grouped",
+                       excess_bar=None)
     assert res["ok"], res
