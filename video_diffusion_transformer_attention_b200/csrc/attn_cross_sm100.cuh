@@ -10,11 +10,14 @@
 // prologue (barrier and TMEM setup, the Q load from HBM, the first product
 // before any softmax can start) and epilogue, with nothing to overlap them.
 // Here a work item is one 128-row query tile, and the kernel is persistent:
-// two CTAs per SM (256 TMEM columns for S and O, 97 KB of shared memory for Q
-// and a two-slot K/V ring, each), each taking items c, c + gridDim.x, ...
+// two CTAs per SM (256 TMEM columns for S and O, 105 KB of shared memory for
+// Q, a two-slot K/V ring and the epilogue's staging, each), each taking items
+// c, c + gridDim.x, ...
 // The next item's Q loads as soon as the current item's last S has read Q,
 // so a CTA's item switch costs no HBM round trip, and the other CTA on the SM
-// fills the tensor core and MUFU while this one is in its epilogue.
+// fills the tensor core and MUFU while this one is in its epilogue.  The
+// epilogue writes O with TMA stores of 32-row boxes staged in shared memory,
+// not with per-thread row stores that touch 32 rows per instruction.
 //
 // Roles (192 threads):
 //   warps 0-3   softmax, correction and epilogue of the query tile

@@ -20,7 +20,14 @@
 //   * P is handed over in two 64-key halves, so O_t += P_t V starts on keys
 //     0-63 while keys 64-127 are still being exponentiated;
 //   * the scale-and-subtract and the row sum run as packed fp32x2 ops, so the
-//     issue slots left over around MUFU ex2 stay free for the other warps.
+//     issue slots left over around MUFU ex2 stay free for the other warps;
+//   * after the first key tile the reference max moves only when a score
+//     exceeds it by more than 2^8 (lazy rescaling), and that is checked
+//     without a full 128-key max: keys 0-63 are exponentiated against the
+//     current reference first, and one of them exceeds it by more than the
+//     threshold only if their exponentials sum to more than 2^8; keys 64-127
+//     are checked by their max.  The exact tile max is taken only when a
+//     check fires.
 //
 // Roles (384 threads, three warpgroups):
 //   warps 0-3   softmax + correction + epilogue of query tile 0
@@ -560,16 +567,36 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 exp_chunk(s[0], scale2, negm2, pa[0], lsum);
                 exp_chunk(s[1], scale2, negm2, pa[1], lsum);
             } else {
-                // Exponentiate keys 0-63 against the current reference while the
-                // tile max is computed alongside; only if the max grew past the
-                // threshold (rare) are O and l rescaled and keys 0-63 redone.
+                // Exponentiate keys 0-63 against the current reference and
+                // store them to TMEM at once (released only after the check);
+                // the check needs no full tile max: a key of 0-63 exceeds the
+                // reference by more than the threshold exactly when its
+                // exponential exceeds 2^threshold, so their sum bounds it, and
+                // keys 64-127 take a max over 64 values.
                 const float m_use0 = (m == -INFINITY) ? 0.0f : m;
                 const uint64_t negm2 = pack_f32x2(-m_use0, -m_use0);
                 exp_chunk(s[0], scale2, negm2, pa[0], lsum);
+                tmem_st16(tS, pa[0]);
                 exp_chunk(s[1], scale2, negm2, pa[1], lsum);
-                const float m_tile = tile_max() * scale_log2;
-                const bool rescale = m_tile > m + kRescaleThreshold;
-                if (__any_sync(0xffffffffu, rescale)) {
+                tmem_st16(tS + 16u, pa[1]);
+                float sum0 = 0.0f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    sum0 += __uint_as_float(uint32_t(lsum[q])) + __uint_as_float(uint32_t(lsum[q] >> 32));
+                float mx[4];
+#pragma unroll
+                for (int g = 4; g < 8; ++g) {
+                    const uint32_t* v = &s[g >> 1][(g & 1) * 16];
+                    float a = fmaxf(__uint_as_float(v[0]), __uint_as_float(v[1]));
+#pragma unroll
+                    for (int i = 2; i < 16; i += 2) a = fmax3(a, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+                    mx[g - 4] = a;
+                }
+                const float m_hi = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * scale_log2;
+                const bool check = sum0 > 256.0f || m_hi > m + kRescaleThreshold;  // 256 = 2^threshold
+                if (__any_sync(0xffffffffu, check)) {
+                    const float m_tile = tile_max() * scale_log2;
+                    const bool rescale = m_tile > m + kRescaleThreshold;
                     float alpha = 1.0f;
                     if (rescale) {
                         alpha = ex2_approx(m - m_tile);
@@ -583,6 +610,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                         exp_chunk(s[0], scale2, negm2b, pa[0], lsum);
                         exp_chunk(s[1], scale2, negm2b, pa[1], lsum);
                     }
+                    // the (possibly redone) keys 0-63 over the speculative store
+                    tmem_st_wait();
+                    tmem_st16(tS, pa[0]);
+                    tmem_st16(tS + 16u, pa[1]);
                     // O_t holds sum_k P_k V_k at the old reference: bring it to
                     // the new one before any of this tile's P is released.
 #pragma unroll 1
@@ -596,9 +627,12 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     }
                 }
             }
-            // release keys 0-63, then exponentiate and release keys 64-127
-            tmem_st16(tS, pa[0]);
-            tmem_st16(tS + 16u, pa[1]);
+            // release keys 0-63 (stored above, or here for the first tile),
+            // then exponentiate and release keys 64-127
+            if (idx == 0) {
+                tmem_st16(tS, pa[0]);
+                tmem_st16(tS + 16u, pa[1]);
+            }
             tmem_st_wait();
             tc_fence_before_sync();
             __syncwarp();
