@@ -283,9 +283,17 @@ def run_vdit(args):
     # FLOPs of one step of the whole problem (every head)
     problem_flops = sum(fl.attn_flops(c, inp_cpu.get("block_mask")) for c in w.calls)
     heads = None
+    H_full = w.calls[0].H
     if args.shard == "heads":
         heads = head_range(w.calls[0].H, world, rank)
         w, inp_cpu = shard_heads(w, inp_cpu, *heads)
+    elif args.heads:
+        # a smaller case of the same kernels and sequence lengths (for
+        # profilers): the first `args.heads` heads of the problem
+        if not 0 < args.heads <= w.calls[0].H:
+            raise SystemExit(f"--heads {args.heads}: the workload has {w.calls[0].H} heads")
+        w, inp_cpu = shard_heads(w, inp_cpu, 0, args.heads)
+        problem_flops = sum(fl.attn_flops(c, inp_cpu.get("block_mask")) for c in w.calls)
     inp = {k: v.to(dev) for k, v in inp_cpu.items()}
     outs = []
     for call in w.calls:
@@ -460,6 +468,7 @@ def run_vdit(args):
                                                        FALLBACK_PEAKS["bf16_tflops_sustained"]))
         peak_burst = dtype_ratio * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
         cross = w.calls[1] if len(w.calls) > 1 else None
+        step_bytes = sum(fl.attn_min_bytes(c) for c in w.calls)
         calls = []
         for i, c in enumerate(w.calls):
             calls.append({"call": c.name, "ms": call_ms[i], "tflops": flops_per_call[i] / (call_ms[i] * 1e-3) / 1e12,
@@ -476,7 +485,8 @@ def run_vdit(args):
                                                                   if args.qknorm else "")
                        + (" [8-bit path: E4M3 + V-Smooth + ExpCast-FP8, quantisation inside the step]"
                           if args.path == "fp8" else ""),
-                       "l2": "inputs larger than L2 (3.1 GB per step)",
+                       "l2": f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB of compulsory traffic per step)",
+                       **({"heads": f"first {args.heads} of {H_full}"} if args.heads and heads is None else {}),
                        "parallelism": (f"heads split over {world} ranks (rank r: heads [r*H/N, (r+1)*H/N) of "
                                        f"the one problem; rank 0 heads {heads[0]}-{heads[1] - 1}), no collective"
                                        if heads is not None else
@@ -716,7 +726,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("vdit", "reference"), default="vdit")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(wl.WORKLOADS))
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--reference-seconds", type=float, default=40.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", choices=("bf16", "fp8"), default="bf16",
@@ -728,6 +738,8 @@ def main():
                          "and the K/V gather")
     ap.add_argument("--clusters", type=int, default=64, help="--kernel group: clusters per head")
     ap.add_argument("--group-iters", type=int, default=1, help="--kernel group: Lloyd iterations")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="compute only the first N heads of each call (a smaller case of the same kernels)")
     ap.add_argument("--shard", choices=("replicas", "heads"), default="replicas",
                     help="N > 1: every rank runs the whole workload (replicas, weak scaling), or the ranks split "
                          "the one problem by heads (strong scaling, no collective)")

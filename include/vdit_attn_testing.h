@@ -40,6 +40,26 @@ vdit_status vdit_testing_attn_fwd(const void* q, const void* k, const void* v,
                                   unsigned long long wait_timeout_ns,
                                   void* stream);
 
+/*
+ * vdit_testing_cross_cta_spans -- the cross-attention call (mask CROSS; same
+ * arguments, rules and outputs as vdit_attn_fwd) that also records, for each
+ * CTA of its persistent grid, the SM it ran on and when its TMA producer
+ * started and finished (%globaltimer, ns).  It exists so a test can see how
+ * many of the kernel's CTAs an SM holds at once, which the occupancy query
+ * does not report correctly for this kernel.
+ *   spans     : device uint64 [max_ctas][3] = {smid, start ns, end ns},
+ *               8-byte aligned; must hold one row per CTA of the grid
+ *   grid_ctas : out, the number of CTAs launched (rows written)
+ * VDIT_ERR_INVALID_ARG if spans or grid_ctas is NULL or max_ctas is smaller
+ * than the grid.  Asynchronous on `stream`.
+ */
+vdit_status vdit_testing_cross_cta_spans(const void* q, const void* k,
+                                         const void* v, void* o, float* lse,
+                                         int B, int H, int Sq, int Skv, int D,
+                                         float scale, unsigned long long* spans,
+                                         int max_ctas, int* grid_ctas,
+                                         void* stream);
+
 #ifdef __cplusplus
 }
 #endif

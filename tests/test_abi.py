@@ -215,3 +215,17 @@ def test_empty_call_is_a_no_op():
     for B, H, Sq in [(0, 2, 64), (1, 0, 64), (1, 2, 0)]:
         assert vb.vdit_attn_fwd(None, None, None, None, None, B, H, Sq, 64, 128, 0.1, 0, 0,
                                 stream=0, check=False) == vb.VDIT_OK
+
+
+def test_cta_span_entry_checks_its_buffer_on_the_host():
+    ok_args = dict(q=1 << 20, k=2 << 20, v=3 << 20, o=4 << 20, lse=None, B=1, H=2, Sq=300, Skv=77, D=128, scale=0.1)
+    a = ok_args
+    st, grid = vb.vdit_testing_cross_cta_spans(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["Sq"],
+                                               a["Skv"], a["D"], a["scale"], None, 16)
+    assert st == vb.VDIT_ERR_INVALID_ARG and grid == 0
+    st, _ = vb.vdit_testing_cross_cta_spans(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["Sq"],
+                                            a["Skv"], a["D"], a["scale"], (5 << 20) + 4, 16)
+    assert st == vb.VDIT_ERR_MISALIGNED
+    st, _ = vb.vdit_testing_cross_cta_spans(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["Sq"],
+                                            a["Skv"], a["D"], a["scale"], 5 << 20, 0)
+    assert st == vb.VDIT_ERR_INVALID_ARG

@@ -108,6 +108,39 @@ def test_cross_attention_over_several_waves(B, H, Sq, Skv):
     compare_all_rows(q, k, v, 1 / math.sqrt(128), CROSS, 0, f"cross {B}x{H}x{Sq}x{Skv}")
 
 
+def test_cross_attention_runs_two_ctas_per_sm():
+    """The persistent cross-attention grid is two CTAs per SM, which the
+    occupancy query does not confirm for this kernel: the CTAs record the SM
+    they ran on and their lifetimes, and every SM must hold two of them at the
+    same time.  The recording call's output is the product call's, bit for bit."""
+    from collections import Counter
+    dev = torch.device("cuda:0")
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    B, H, Sq, Skv = 1, 40, 20000, 512
+    q, k, v = (t.to(dev) for t in wl.draw_qkv(B, H, Sq, Skv, 128, seed=43, recipe="rms_qk"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Sq), dtype=torch.float32, device=dev)
+    spans = torch.zeros((4 * sms, 3), dtype=torch.int64, device=dev)
+    st, grid = vb.vdit_testing_cross_cta_spans(q, k, v, o, lse, B, H, Sq, Skv, 128, 1 / math.sqrt(128), spans,
+                                               4 * sms)
+    assert st == vb.VDIT_OK, vb.vdit_status_string(st)
+    assert vb.vdit_get_device_status()[0] == vb.VDIT_OK
+    assert grid == 2 * sms
+    all_rows = spans.cpu().numpy()
+    assert (all_rows[grid:] == 0).all()  # one row per launched CTA, no more
+    sp = all_rows[:grid]
+    smid, t0, t1 = sp[:, 0], sp[:, 1], sp[:, 2]
+    assert (t1 > t0).all()
+    per_sm = Counter(smid.tolist())
+    assert len(per_sm) == sms and set(per_sm.values()) == {2}
+    for s in per_sm:
+        a, b = np.nonzero(smid == s)[0]
+        assert max(t0[a], t0[b]) < min(t1[a], t1[b]), f"SM {s}: the two CTAs did not run at the same time"
+    o2, l2 = vb.attention(q, k, v, None, CROSS, 0)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(lse, l2)
+
+
 def test_cross_attention_is_deterministic():
     dev = torch.device("cuda:0")
     q, k, v = (t.to(dev) for t in wl.draw_qkv(1, 8, 20000, 512, 128, seed=42, recipe="rms_qk"))

@@ -56,6 +56,7 @@ EXPORTS = (
     "vdit_status_string",
     "vdit_abi_version",
     "vdit_testing_attn_fwd",
+    "vdit_testing_cross_cta_spans",
 )
 
 _lock = threading.Lock()
@@ -123,6 +124,9 @@ def lib() -> ctypes.CDLL:
             h.vdit_attn_merge_f32.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, vp]
             h.vdit_testing_attn_fwd.restype = c_int
             h.vdit_testing_attn_fwd.argtypes = fwd_args + [c_int, ctypes.c_ulonglong, vp]
+            h.vdit_testing_cross_cta_spans.restype = c_int
+            h.vdit_testing_cross_cta_spans.argtypes = [vp] * 5 + [c_int] * 5 + [c_float, vp, c_int,
+                                                                              ctypes.POINTER(c_int), vp]
             h.vdit_get_device_status.restype = c_int
             h.vdit_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
             h.vdit_status_string.restype = ctypes.c_char_p
@@ -382,6 +386,16 @@ def vdit_testing_attn_fwd(q, k, v, o, lse, B, H, Sq, Skv, D, scale, mask_kind, c
     return int(lib().vdit_testing_attn_fwd(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), B, H, Sq, Skv, D,
                                            float(scale), mask_kind, chunk_tokens, int(fault),
                                            int(wait_timeout_ns), _stream(stream)))
+
+
+def vdit_testing_cross_cta_spans(q, k, v, o, lse, B, H, Sq, Skv, D, scale, spans, max_ctas, stream=None):
+    """Test-only cross-attention call recording each CTA's (smid, start ns, end ns) into spans
+    (see include/vdit_attn_testing.h); returns (status, CTAs launched)."""
+    grid = ctypes.c_int(0)
+    st = lib().vdit_testing_cross_cta_spans(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), B, H, Sq, Skv, D,
+                                            float(scale), _addr(spans), int(max_ctas), ctypes.byref(grid),
+                                            _stream(stream))
+    return int(st), int(grid.value)
 
 
 def vdit_get_device_status(stream=None):

@@ -10,14 +10,15 @@
 // prologue (barrier and TMEM setup, the Q load from HBM, the first product
 // before any softmax can start) and epilogue, with nothing to overlap them.
 // Here a work item is one 128-row query tile, and the kernel is persistent:
-// two CTAs per SM (256 TMEM columns for S and O, 105 KB of shared memory for
-// Q, a two-slot K/V ring and the epilogue's staging, each), each taking items
-// c, c + gridDim.x, ...
+// two CTAs per SM (256 TMEM columns for S and O, 97 KB of shared memory for Q
+// and a two-slot K/V ring, each), each taking items c, c + gridDim.x, ...
 // The next item's Q loads as soon as the current item's last S has read Q,
 // so a CTA's item switch costs no HBM round trip, and the other CTA on the SM
 // fills the tensor core and MUFU while this one is in its epilogue.  The
-// epilogue writes O with TMA stores of 32-row boxes staged in shared memory,
-// not with per-thread row stores that touch 32 rows per instruction.
+// epilogue stages O in the V slot (free once the item's last P V is done) and
+// writes it with TMA stores of 32-row boxes, not with per-thread row stores
+// that touch 32 rows per instruction; the producer loads the next item's first
+// V only after those stores have read the slot.
 //
 // Roles (192 threads):
 //   warps 0-3   softmax, correction and epilogue of the query tile
@@ -58,19 +59,19 @@ struct __align__(8) CrossBarriers {
     uint64_t s_full;
     uint64_t p_full[2];    // P keys 0-63 / 64-127 in TMEM
     uint64_t o_full;
+    uint64_t stage_free;   // the epilogue's TMA stores have read the V slot it staged O in
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
 };
 
-constexpr int kCrossStageRows = 32;   // epilogue: one warp's rows
-constexpr int kCrossStageCols = 32;   // head dims per staged chunk (64 bytes of a bf16 row)
-constexpr int kCrossStageBytes = kCrossStageRows * kCrossStageCols * 2;  // 2 KB per softmax warp
+constexpr int kCrossStageRows = 32;  // epilogue: one warp's rows, staged in the V slot
+constexpr int kCrossStageCols = 64;  // head dims per TMA store box (128 bytes of a bf16 row, 128B-swizzled)
+constexpr int kCrossStageBytes = kCrossStageRows * kHeadDim * 2;  // 8 KB per softmax warp: two boxes
 
 constexpr int kCrossSmemQ = 0;
 constexpr int kCrossSmemKV = kTileBytes;
-constexpr int kCrossSmemStage = kCrossSmemKV + 2 * kTileBytes;  // 4 x 2 KB: the epilogue's store staging
-constexpr int kCrossSmemBar = kCrossSmemStage + 4 * kCrossStageBytes;
+constexpr int kCrossSmemBar = kCrossSmemKV + 2 * kTileBytes;
 constexpr int kCrossSmemBytes = kCrossSmemBar + ((int(sizeof(CrossBarriers)) + 15) / 16) * 16 + 1024;  // + alignment
 
 // Item i is query tile i % n_qb of (batch, head) i / n_qb: the CTAs running at
@@ -82,12 +83,20 @@ __device__ __forceinline__ void cross_item(const FwdParams& p, long long item, i
     b = static_cast<int>(bh / p.H);
 }
 
-// tm_o: O as the same 4-D tensor as Q, with 32-dim x 32-row boxes and no
-// swizzle: the epilogue's TMA store unit.
+// Test-only residency record: when `spans` is non-null, CTA c < max_ctas
+// writes spans[3c] = its SM id, spans[3c+1] / spans[3c+2] = the global timer
+// (ns) when its producer starts and finishes.  Null in every product call.
+struct CrossSpans {
+    unsigned long long* spans;
+    int max_ctas;
+};
+
+// tm_o: O as the same 4-D tensor as Q, with 64-dim x 32-row boxes, 128-byte
+// swizzled: the epilogue's TMA store unit.
 __global__ void __launch_bounds__(kCrossThreads, 2)
     attn_cross_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                            const FwdParams p) {
+                            const FwdParams p, const CrossSpans rec) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw_base + 1023u) & ~1023u) - raw_base);
@@ -109,6 +118,7 @@ __global__ void __launch_bounds__(kCrossThreads, 2)
         }
         mbar_init(smem_addr(&bars->s_full), 1);
         mbar_init(smem_addr(&bars->o_full), 1);
+        mbar_init(smem_addr(&bars->stage_free), 4);  // one elected arrive per softmax warp
         mbar_init(smem_addr(&bars->drain), 1);
         bars->abort = 0;
         fence_barrier_init();
@@ -134,6 +144,16 @@ __global__ void __launch_bounds__(kCrossThreads, 2)
         if (warp == kCrossLoadWarp && lane == 0) {
             // ------------------------------------------------ TMA producer
             griddep_wait();  // Q/K written by a preceding kernel (fused Q/K norm) are complete
+            // test-only: the SM this CTA runs on and its producer's lifetime
+            unsigned long long* span = (rec.spans != nullptr && int(blockIdx.x) < rec.max_ctas)
+                                           ? rec.spans + 3 * size_t(blockIdx.x)
+                                           : nullptr;
+            if (span != nullptr) {
+                uint32_t smid;
+                asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+                span[0] = smid;
+                span[1] = global_timer_ns();
+            }
             uint32_t kt = 0;  // key tiles loaded by earlier items: each used slot 0 (K) and slot 1 (V) once
             uint32_t qi = 0;  // earlier items (only the parities of these counters matter)
             bool ok = true;
@@ -157,6 +177,13 @@ __global__ void __launch_bounds__(kCrossThreads, 2)
                             ok = false;
                             break;
                         }
+                        // the previous item's epilogue staged O in the V slot
+                        if (slot == 1 && j == 0 && qi > 0 &&
+                            !bounded_wait(smem_addr(&bars->stage_free), (qi - 1u) & 1u, abort_flag, p.timeout_ns,
+                                          kSiteProducer)) {
+                            ok = false;
+                            break;
+                        }
                         const uint32_t full = smem_addr(&bars->kv_full[slot]);
                         const CUtensorMap* map = slot ? &tm_v : &tm_k;
                         mbar_arrive_expect_tx(full, kTileBytes);
@@ -166,6 +193,7 @@ __global__ void __launch_bounds__(kCrossThreads, 2)
                 }
                 kt += uint32_t(n_kv);
             }
+            if (span != nullptr) span[2] = global_timer_ns();
         } else if (warp == kCrossMmaWarp && lane == 0) {
             // ------------------------------------------------ MMA issuer
             const uint32_t tS = tmem;
@@ -337,14 +365,17 @@ __global__ void __launch_bounds__(kCrossThreads, 2)
                 const int row = q0 + row_in_tile;
                 const int warp_row0 = q0 + warp * kCrossStageRows;  // first row of this warp's TMA boxes
                 const float inv_l = 1.0f / l;  // l >= 1: the row's maximum key contributes 2^0
-                // O leaves through shared memory, 32 head dims at a time: each
-                // thread writes its row's 64 bytes into the warp's 2 KB staging
-                // box, and one TMA store moves the 32 x 32 box to global memory,
+                // O leaves through shared memory: each thread writes its row
+                // (256 bytes) into the warp's 8 KB of the V slot -- free once
+                // the item's last P V has completed -- as two 128B-swizzled
+                // 32-row x 64-dim boxes, and one lane stores both with TMA
                 // instead of 32 rows of 16-byte pieces per store instruction.
-                uint8_t* stage = smem + kCrossSmemStage + warp * kCrossStageBytes;
+                uint8_t* stage = smem + kCrossSmemKV + kTileBytes + warp * kCrossStageBytes;
                 const uint32_t stage_addr = smem_addr(stage);
-#pragma unroll
-                for (int c = 0; c < kHeadDim / kCrossStageCols; ++c) {
+                uint8_t* my_row = stage + lane * 128;
+                const uint32_t swz = uint32_t(lane & 7) << 4;  // 128-byte swizzle: 16-byte chunk ^= row % 8
+#pragma unroll 1
+                for (int c = 0; c < kHeadDim / 32; ++c) {
                     uint32_t o[32];
                     tmem_ld32(tO + uint32_t(c) * 32u, o);
                     tmem_ld_wait(o);
@@ -352,18 +383,23 @@ __global__ void __launch_bounds__(kCrossThreads, 2)
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
                         pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-                    // the previous box's store has read the staging buffer
-                    if (lane == 0) bulk_wait_read_all();
-                    __syncwarp();
-                    uint4* dst = reinterpret_cast<uint4*>(stage + lane * (kCrossStageCols * 2));
+                    // dims 32c .. 32c+31: box c / 2, 16-byte chunks 4 (c % 2) + i of the row
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0 && warp_row0 < p.Sq) {
-                        tma_store_4d(&tm_o, stage_addr, c * kCrossStageCols, h, warp_row0, b);
+                    for (int i = 0; i < 4; ++i)
+                        *reinterpret_cast<uint4*>(my_row + (c >> 1) * (kCrossStageBytes / 2) +
+                                                  ((uint32_t((4 * (c & 1) + i) << 4)) ^ swz)) =
+                            make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    if (warp_row0 < p.Sq) {
+                        tma_store_4d(&tm_o, stage_addr, 0, h, warp_row0, b);
+                        tma_store_4d(&tm_o, stage_addr + kCrossStageBytes / 2, kCrossStageCols, h, warp_row0, b);
                         bulk_commit_group();
+                        bulk_wait_read_all();  // the boxes have left shared memory
                     }
+                    mbar_arrive(smem_addr(&bars->stage_free));
                 }
                 if (p.lse != nullptr && row < p.Sq)
                     p.lse[(static_cast<size_t>(b) * p.H + h) * p.Sq + row] = (m + __log2f(l)) * 0.69314718055994531f;

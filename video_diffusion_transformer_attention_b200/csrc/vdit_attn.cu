@@ -164,8 +164,8 @@ bool encode_bshd(CUtensorMap* map, const void* base, int B, int S, int H) {
 }
 
 // The output O as a store target for the cross-attention epilogue: the same
-// 4-D view, boxes of 32 head dims x 32 tokens, no swizzle (a warp's rows, one
-// 64-byte piece each).  Rows past S are not written.
+// 4-D view, boxes of 64 head dims x 32 tokens (a warp's rows, 128 bytes each),
+// 128-byte swizzled.  Rows past S are not written.
 bool encode_bshd_store(CUtensorMap* map, void* base, int B, int S, int H) {
     PFN_cuTensorMapEncodeTiled_v12000 f = encode_fn();
     if (f == nullptr) return false;
@@ -175,13 +175,13 @@ bool encode_bshd_store(CUtensorMap* map, void* base, int B, int S, int H) {
     cuuint32_t box[4] = {cuuint32_t(vdit::kCrossStageCols), 1, cuuint32_t(vdit::kCrossStageRows), 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     return f(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 vdit_status launch(const void* q, const void* k, const void* v, void* o, float* lse, const uint8_t* block_mask,
                    const Shape& s, float scale, int debug_flags, unsigned long long timeout_ns, cudaStream_t stream,
-                   bool after_norm) {
+                   bool after_norm, unsigned long long* cta_spans = nullptr, int max_span_ctas = 0) {
     int dev = 0;
     const DeviceState* ds = nullptr;
     vdit_status st = ensure_device(&dev, &ds);
@@ -211,9 +211,10 @@ vdit_status launch(const void* q, const void* k, const void* v, void* o, float* 
         const dim3 grid(static_cast<unsigned>(items < ds->cross_grid ? items : ds->cross_grid));
         CUtensorMap to;
         if (!encode_bshd_store(&to, o, s.B, s.Sq, s.H)) return VDIT_ERR_CUDA;
+        const vdit::CrossSpans rec{cta_spans, max_span_ctas};
         if (!after_norm) {
             vdit::attn_cross_sm100_kernel<<<grid, vdit::kCrossThreads, vdit::kCrossSmemBytes, stream>>>(tq, tk, tv, to,
-                                                                                                      p);
+                                                                                                      p, rec);
             return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
         }
         cudaLaunchConfig_t cfg{};
@@ -226,7 +227,7 @@ vdit_status launch(const void* q, const void* k, const void* v, void* o, float* 
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, vdit::attn_cross_sm100_kernel, tq, tk, tv, to, p) == cudaSuccess
+        return cudaLaunchKernelEx(&cfg, vdit::attn_cross_sm100_kernel, tq, tk, tv, to, p, rec) == cudaSuccess
                    ? VDIT_OK
                    : VDIT_ERR_CUDA;
     }
@@ -261,7 +262,8 @@ vdit_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
                      int Skv, int D, float scale, int mask_kind, int chunk_tokens, void* workspace,
                      size_t workspace_bytes, void* stream, int debug_flags = 0,
                      unsigned long long timeout_ns = kDefaultWaitTimeoutNs,
-                     const uint8_t* block_mask = nullptr, bool after_norm = false) {
+                     const uint8_t* block_mask = nullptr, bool after_norm = false,
+                     unsigned long long* cta_spans = nullptr, int max_span_ctas = 0) {
     (void)workspace;
     (void)workspace_bytes;  // no shape needs a workspace in this version
     const Shape s{B, H, Sq, Skv, D, mask_kind, chunk_tokens};
@@ -291,7 +293,7 @@ vdit_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
             return VDIT_ERR_INVALID_ARG;
     }
     return launch(q, k, v, o, lse, block_mask, s, scale, debug_flags, timeout_ns, static_cast<cudaStream_t>(stream),
-                  after_norm);
+                  after_norm, cta_spans, max_span_ctas);
 }
 
 // ------------------------------------------------------------ Q/K RMS norm
@@ -928,6 +930,33 @@ vdit_status vdit_testing_attn_fwd(const void* q, const void* k, const void* v, v
         const int flags = fault == VDIT_TESTING_WITHHOLD_KV ? vdit::kDebugWithholdKV : 0;
         return fwd_impl(q, k, v, o, lse, B, H, Sq, Skv, D, scale, mask_kind, chunk_tokens, nullptr, 0, stream, flags,
                         wait_timeout_ns);
+    } catch (...) {
+        return VDIT_ERR_CUDA;
+    }
+}
+
+vdit_status vdit_testing_cross_cta_spans(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                                         int H, int Sq, int Skv, int D, float scale, unsigned long long* spans,
+                                         int max_ctas, int* grid_ctas, void* stream) {
+    try {
+        if (spans == nullptr || max_ctas < 1 || grid_ctas == nullptr) return VDIT_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(spans) & 7u) != 0) return VDIT_ERR_MISALIGNED;
+        *grid_ctas = 0;
+        const Shape s{B, H, Sq, Skv, D, VDIT_MASK_CROSS, 0};
+        vdit_status st = check_shape(s, true, scale);
+        if (st != VDIT_OK) return st;
+        if (B == 0 || H == 0 || Sq == 0) return VDIT_OK;
+        int dev = 0;
+        const DeviceState* ds = nullptr;
+        st = ensure_device(&dev, &ds);
+        if (st != VDIT_OK) return st;
+        const long long items = static_cast<long long>(cross_tiles(Sq)) * H * B;
+        const int grid = static_cast<int>(items < ds->cross_grid ? items : ds->cross_grid);
+        if (grid > max_ctas) return VDIT_ERR_INVALID_ARG;  // every CTA records its span
+        st = fwd_impl(q, k, v, o, lse, B, H, Sq, Skv, D, scale, VDIT_MASK_CROSS, 0, nullptr, 0, stream, 0,
+                      kDefaultWaitTimeoutNs, nullptr, false, spans, max_ctas);
+        if (st == VDIT_OK) *grid_ctas = grid;
+        return st;
     } catch (...) {
         return VDIT_ERR_CUDA;
     }
