@@ -428,18 +428,24 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             // that tile's P V on e comes its S on its next entry (two entries
             // on while both lists last, then the next one), so the two tiles
             // keep taking turns.  Barrier phases count each tile's own entries.
-            auto owner = [&](int e) -> int { return (kv_list[e] >> 14) & 1; };
+            // The stream's shape follows from the two list lengths alone
+            // (sparse_pos): entries [0, both2) alternate between the tiles,
+            // the rest belong to the tile with the longer list.  Owner and
+            // next entry are register arithmetic, no shared-memory reads.
+            const int n0 = kv_list_len[1], n1 = kv_list_len[2];
+            const int both2 = 2 * min(n0, n1);
+            const int lt = n0 >= n1 ? 0 : 1;
+            auto owner = [&](int e) -> int { return e < both2 ? (e & 1) : lt; };
             auto next_own = [&](int e) -> int {  // the owner's next entry after e, or -1
-                const int t = owner(e);
-                for (int f = e + 1; f < n_kv; ++f)
-                    if (owner(f) == t) return f;
-                return -1;
+                if (e + 2 < both2) return e + 2;
+                if (e < both2) return ((e & 1) == lt && both2 < n_kv) ? both2 : -1;
+                return e + 1 < n_kv ? e + 1 : -1;
             };
             int done0 = 0, done1 = 0;  // P V products issued per tile (scalars: no local-memory array)
             // prologue: the scores of each tile's first entry (entries 0 and 1
             // while both tiles have entries)
             for (int e = 0; ok && e < 2 && e < n_kv; ++e) {
-                if (e == 1 && owner(1) == owner(0)) break;
+                if (e == 1 && both2 == 0) break;
                 ok = bounded_wait(smem_addr(&bars->kv_full[(2 * e) % kStages]), 0, abort_flag, p.timeout_ns, kSiteMma);
                 if (!ok) break;
                 tc_fence_after_sync();
@@ -470,7 +476,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 const int f = next_own(e);
                 if (f < 0) {
                     umma_commit(smem_addr(&bars->o_full[t]));
-                } else if (f > 1 || owner(1) == owner(0)) {  // entries 0 and 1 of two tiles had theirs in the prologue
+                } else if (f > 1 || both2 == 0) {  // entries 0 and 1 of two tiles had theirs in the prologue
                     const int uk = 2 * f;
                     const int k_slot = uk % kStages;
                     ok = bounded_wait(smem_addr(&bars->kv_full[k_slot]), uint32_t(uk / kStages) & 1u, abort_flag,

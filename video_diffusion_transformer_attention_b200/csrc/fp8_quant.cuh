@@ -139,14 +139,18 @@ __device__ __forceinline__ void stage_v_block(const __nv_bfloat16* __restrict__ 
     for (int r = 0; r < kRows; ++r) reinterpret_cast<uint2*>(tile + (warp + r * (kQuantThreads / 32)) * 128)[lane] = x[r];
 }
 
-// One CTA (256 threads) per (b, h, block); after staging, thread d < 128 owns
-// channel d: block mean (sequential fp32 sum over the block's tokens, then
-// / n), the block's largest |v - mean|, and the running per-channel maxima
-// over the head's blocks (atomicMax on the bits of non-negative floats,
-// which order like the floats).
+// One CTA (256 threads) per (b, h, block); after staging, thread d < 128
+// takes the block mean of channel d (a sequential fp32 sum over the block's
+// tokens, then / n: one dependent chain per channel, in token order), and
+// both halves of the CTA then take the largest |v - mean| of channel d over
+// tokens 0-63 and 64-127 (a max, exact in any order), combined through shared
+// memory.  Thread d < 128 then updates the running per-channel maxima over
+// the head's blocks (atomicMax on the bits of non-negative floats, which
+// order like the floats).
 __global__ void __launch_bounds__(kQuantThreads)
     v_stats_kernel(const __nv_bfloat16* __restrict__ v, Fp8Tensors t, int B, int H, int Skv) {
     __shared__ __align__(16) __nv_bfloat16 tile[kQuantBlock * 128];
+    __shared__ float mu_s[128], rmax_s[128];
     const int nkb = (Skv + kQuantBlock - 1) / kQuantBlock;
     const int blk = blockIdx.x % nkb;
     const int h = (blockIdx.x / nkb) % H;
@@ -155,25 +159,42 @@ __global__ void __launch_bounds__(kQuantThreads)
     const int n = min(kQuantBlock, Skv - t0);
     stage_v_block(v, tile, b, h, H, Skv, t0, n);
     __syncthreads();
-    const int d = threadIdx.x;
-    if (d >= 128) return;
-    float sum = 0.0f;
-    for (int i = 0; i < n; ++i) sum += __bfloat162float(tile[i * 128 + d]);
-    const float mu = sum / static_cast<float>(n);
+    const int d = threadIdx.x & 127;
+    const int half = threadIdx.x >> 7;
+    if (half == 0) {
+        float sum = 0.0f;
+        if (n == kQuantBlock) {
+#pragma unroll 16
+            for (int i = 0; i < kQuantBlock; ++i) sum += __bfloat162float(tile[i * 128 + d]);
+        } else {
+            for (int i = 0; i < n; ++i) sum += __bfloat162float(tile[i * 128 + d]);
+        }
+        mu_s[d] = sum / static_cast<float>(n);
+    }
+    __syncthreads();
+    const float mu = mu_s[d];
+    const int i1 = min(n, (half + 1) * (kQuantBlock / 2));
     float rmax = 0.0f;
-    for (int i = 0; i < n; ++i) rmax = fmaxf(rmax, fabsf(__bfloat162float(tile[i * 128 + d]) - mu));
-    const size_t bh = static_cast<size_t>(b) * H + h;
-    t.mu[(bh * nkb + blk) * 128 + d] = mu;
-    atomicMax(t.v_amax_r + bh * 128 + d, __float_as_uint(rmax));
-    atomicMax(t.v_amax_mu + bh * 128 + d, __float_as_uint(fabsf(mu)));
+#pragma unroll 8
+    for (int i = half * (kQuantBlock / 2); i < i1; ++i)
+        rmax = fmaxf(rmax, fabsf(__bfloat162float(tile[i * 128 + d]) - mu));
+    if (half == 1) rmax_s[d] = rmax;
+    __syncthreads();
+    if (half == 0) {
+        rmax = fmaxf(rmax, rmax_s[d]);
+        const size_t bh = static_cast<size_t>(b) * H + h;
+        t.mu[(bh * nkb + blk) * 128 + d] = mu;
+        atomicMax(t.v_amax_r + bh * 128 + d, __float_as_uint(rmax));
+        atomicMax(t.v_amax_mu + bh * 128 + d, __float_as_uint(fabsf(mu)));
+    }
 }
 
-// One CTA (256 threads) per (b, h, block).  After staging, thread d < 128
-// computes the residual codes E4M3((v - mean) * 448 / amax_d) of channel d
-// into a transposed shared-memory tile ([channel][token] bytes), which the
-// whole CTA then writes out as contiguous 16-byte rows; threads 128-255 write
-// the block's restore tile meanwhile (rows 3-15 zero as 16-byte stores, rows
-// 0-2 one bf16 per thread).
+// One CTA (256 threads) per (b, h, block).  After staging, threads d and
+// d + 128 compute the residual codes E4M3((v - mean) * 448 / amax_d) of
+// channel d, four 16-token groups each, into a transposed shared-memory tile
+// ([channel][token] bytes), which the whole CTA then writes out as
+// contiguous 16-byte rows; the block's restore tile (rows 3-15 zero as
+// 16-byte stores, rows 0-2 one bf16 per thread) is written in between.
 __global__ void __launch_bounds__(kQuantThreads)
     v_quant_kernel(const __nv_bfloat16* __restrict__ v, Fp8Tensors t, int B, int H, int Skv) {
     __shared__ __align__(16) __nv_bfloat16 tile[kQuantBlock * 128];
@@ -193,13 +214,15 @@ __global__ void __launch_bounds__(kQuantThreads)
                              __uint_as_float(t.v_amax_mu[bh * 128 + d]) * kMuFloor);
     const float inv = amax > 0.0f ? kE4M3Max / amax : 0.0f;
     const float mu = t.mu[(bh * nkb + blk) * 128 + d];
-    if (threadIdx.x < 128) {
-        if (blk == 0) t.v_scale[bh * 128 + d] = amax / kE4M3Max;
-        // 16 tokens per 16-byte word; the word index is rotated by the channel so
-        // that the 32 lanes of a warp store to different banks
+    const int hsel = threadIdx.x >> 7;
+    if (hsel == 0 && blk == 0) t.v_scale[bh * 128 + d] = amax / kE4M3Max;
+    {
+        // 16 tokens per 16-byte word; half hsel takes the words of parity
+        // hsel, rotated by the channel so that a warp's 16-byte stores spread
+        // over the banks
 #pragma unroll 1
-        for (int gi = 0; gi < 8; ++gi) {
-            const int g = (gi + (d >> 2)) & 7;
+        for (int gi = 0; gi < 4; ++gi) {
+            const int g = (2 * (gi + (d >> 2)) + hsel) & 7;
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -213,12 +236,13 @@ __global__ void __launch_bounds__(kQuantThreads)
             }
             reinterpret_cast<uint4*>(codes + d * kQuantBlock)[g] = make_uint4(w[0], w[1], w[2], w[3]);
         }
-    } else {
-        // zero rows 3-15 of both halves: 2 x 13 rows x 8 chunks of 16 bytes
-        for (int i = threadIdx.x - 128; i < 2 * 13 * 8; i += 128) {
-            const int half = i / (13 * 8), r = 3 + (i / 8) % 13, ch = i % 8;
-            *reinterpret_cast<uint4*>(img + half * 2048 + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
-        }
+    }
+    // zero rows 3-15 of both halves: 2 x 13 rows x 8 chunks of 16 bytes
+    for (int i = threadIdx.x; i < 2 * 13 * 8; i += kQuantThreads) {
+        const int half = i / (13 * 8), r = 3 + (i / 8) % 13, ch = i % 8;
+        *reinterpret_cast<uint4*>(img + half * 2048 + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+    }
+    if (hsel == 1) {
         // Restore tile: element (row k, channel d) of half d / 64 at
         // k * 128 + ((c / 8) ^ (k & 7)) * 16 + (c % 8) * 2, c = d % 64.
         const float mu_p = mu * inv;
