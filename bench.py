@@ -87,6 +87,49 @@ def workload_config(name):
     return w, desc
 
 
+# head axis of each input tensor: BSHD tensors on axis 2, the block mask
+# [B, H, n_qb, n_kvb] on axis 1
+HEAD_AXIS = {"q": 2, "k": 2, "v": 2, "k_text": 2, "v_text": 2, "block_mask": 1}
+
+
+def cudart():
+    """The CUDA runtime already loaded by torch (for pitched async copies)."""
+    import ctypes
+    for name in ("libcudart.so.12", "/usr/local/cuda/lib64/libcudart.so.12"):
+        try:
+            rt = ctypes.CDLL(name)
+        except OSError:
+            continue
+        rt.cudaMemcpy2DAsync.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_size_t,
+                                         ctypes.c_size_t, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p]
+        rt.cudaMemcpy2DAsync.restype = ctypes.c_int
+        return rt
+    raise SystemExit("libcudart.so.12 not found")
+
+
+def copy_heads(rt, dev_t, host_t, axis, h0, hg, upload, stream):
+    """Copy heads [h0, h0 + hg) between a pinned host tensor holding every
+    head and a compact device tensor holding only those heads, as one
+    pitched copy: rows are the dims before the head axis, each row's
+    segment the hg heads' contiguous bytes."""
+    es = host_t.element_size()
+    inner = es
+    for n in host_t.shape[axis + 1:]:
+        inner *= n
+    rows = 1
+    for n in host_t.shape[:axis]:
+        rows *= n
+    H = host_t.shape[axis]
+    width, pitch = hg * inner, H * inner
+    host_ptr = host_t.data_ptr() + h0 * inner
+    if upload:
+        err = rt.cudaMemcpy2DAsync(dev_t.data_ptr(), width, host_ptr, pitch, width, rows, 1, stream.cuda_stream)
+    else:
+        err = rt.cudaMemcpy2DAsync(host_ptr, pitch, dev_t.data_ptr(), width, width, rows, 2, stream.cuda_stream)
+    if err != 0:
+        raise SystemExit(f"cudaMemcpy2DAsync failed ({err})")
+
+
 def call_inputs(inp, call):
     if call.mask_kind == wl.MASK_CROSS:
         return inp["q"], inp["k_text"], inp["v_text"]
@@ -323,7 +366,7 @@ def run_vdit(args):
     launches_per_call = [(4 if args.path == "fp8" else 1) + (1 if args.qknorm and c.name == "self" else 0)
                          for c in w.calls]
 
-    def launch(i, call, q, k, v, o, lse, mid_event=None):
+    def launch(i, call, q, k, v, o, lse, mid_event=None, mask=None):
         if args.path == "fp8":
             # quantise (one memset + three kernels), then the 8-bit attention
             ws = fp8_ws[i]
@@ -337,8 +380,8 @@ def run_vdit(args):
                                     call.D, call.scale, call.mask_kind, call.chunk_tokens, qk_ws, qk_ws.numel(),
                                     sptr)
         elif call.mask_kind == wl.MASK_BLOCK_SPARSE:
-            vb.vdit_attn_fwd_block_sparse(q, k, v, o, lse, inp["block_mask"], call.B, call.H, call.Sq, call.Skv,
-                                          call.D, call.scale, sptr)
+            vb.vdit_attn_fwd_block_sparse(q, k, v, o, lse, inp["block_mask"] if mask is None else mask, call.B,
+                                          call.H, call.Sq, call.Skv, call.D, call.scale, sptr)
         else:
             vb.vdit_attn_fwd(q, k, v, o, lse, call.B, call.H, call.Sq, call.Skv, call.D, call.scale,
                              call.mask_kind, call.chunk_tokens, sptr)
@@ -396,45 +439,70 @@ def run_vdit(args):
     value = job_tflops(1, job_step_flops, args.steps, ms_max)
 
     # ---- end to end through the public API, host buffers in and out
-    # Every step copies its inputs from pinned host memory and its results back.
-    # Three streams pipeline consecutive steps over two device buffer sets:
-    # while step i computes, step i+1's inputs go up and step i-1's results
-    # come down (separate copy engines, each direction at full PCIe rate).
+    # Every step copies its inputs from pinned host memory and its results
+    # back.  The heads are split into G groups (heads are independent): each
+    # group's Q/K/V go up as one pitched copy per tensor into compact
+    # [B, S, H/G, D] device buffers, the group's calls run as soon as its
+    # inputs have landed, and its O/LSE go down while the next group
+    # computes.  Across steps, two device buffer sets and three streams let
+    # step i+1's uploads and step i-1's downloads run during step i.  Only
+    # the first group's upload and the last group's download are exposed.
     e2e = None
     if args.e2e_steps > 0:
+        import dataclasses
+        H = w.calls[0].H
+        # the largest group count up to the requested one that divides H
+        G = max(g for g in range(1, max(1, args.e2e_head_groups) + 1) if H % g == 0)
+        hg = H // G
+        rt = cudart()
         host_in = {k: v.pin_memory() for k, v in inp_cpu.items()}
         host_out = [(torch.empty(o.shape, dtype=o.dtype).pin_memory(), torch.empty(l.shape, dtype=l.dtype).pin_memory())
                     for o, l in outs]
         h2d = sum(t.numel() * t.element_size() for t in host_in.values())
         d2h = sum(o.numel() * o.element_size() + l.numel() * l.element_size() for o, l in host_out)
-        inp_sets = [inp, {k: torch.empty_like(v) for k, v in inp.items()}]
-        out_sets = [outs, [(torch.empty_like(o), torch.empty_like(l)) for o, l in outs]]
+        gcalls = [dataclasses.replace(c, H=hg) for c in w.calls]
+
+        def group_shape(t, axis):
+            return tuple(hg if a == axis else n for a, n in enumerate(t.shape))
+
+        # [buffer set][group] -> device tensors
+        g_in = [[{k: torch.empty(group_shape(v, HEAD_AXIS[k]), dtype=v.dtype, device=dev) for k, v in inp.items()}
+                 for _ in range(G)] for _ in range(2)]
+        g_out = [[[(torch.empty(group_shape(o, 2), dtype=o.dtype, device=dev),
+                    torch.empty(group_shape(l, 1), dtype=l.dtype, device=dev)) for o, l in outs]
+                  for _ in range(G)] for _ in range(2)]
         s_in = torch.cuda.Stream(device=dev)
         s_out = torch.cuda.Stream(device=dev)
-        ev = {name: [torch.cuda.Event() for _ in range(2)] for name in ("in_ready", "in_free", "out_ready", "out_free")}
+        ev_in_ready = [[torch.cuda.Event() for _ in range(G)] for _ in range(2)]
+        ev_out_ready = [[torch.cuda.Event() for _ in range(G)] for _ in range(2)]
+        ev_in_free = [torch.cuda.Event() for _ in range(2)]
+        ev_out_free = [torch.cuda.Event() for _ in range(2)]
 
         def pipelined(n_steps):
             for i in range(n_steps):
                 b = i % 2
                 if i >= 2:
-                    s_in.wait_event(ev["in_free"][b])
-                with torch.cuda.stream(s_in):
+                    s_in.wait_event(ev_in_free[b])
+                for g in range(G):
                     for k_, v_ in host_in.items():
-                        inp_sets[b][k_].copy_(v_, non_blocking=True)
-                ev["in_ready"][b].record(s_in)
-                stream.wait_event(ev["in_ready"][b])
+                        copy_heads(rt, g_in[b][g][k_], v_, HEAD_AXIS[k_], g * hg, hg, True, s_in)
+                    ev_in_ready[b][g].record(s_in)
                 if i >= 2:
-                    stream.wait_event(ev["out_free"][b])
-                with torch.cuda.stream(stream):
-                    step(inp_set=inp_sets[b], out_set=out_sets[b])
-                ev["in_free"][b].record(stream)
-                ev["out_ready"][b].record(stream)
-                s_out.wait_event(ev["out_ready"][b])
-                with torch.cuda.stream(s_out):
-                    for (o, l), (ho, hl) in zip(out_sets[b], host_out):
-                        ho.copy_(o, non_blocking=True)
-                        hl.copy_(l, non_blocking=True)
-                ev["out_free"][b].record(s_out)
+                    stream.wait_event(ev_out_free[b])
+                for g in range(G):
+                    stream.wait_event(ev_in_ready[b][g])
+                    with torch.cuda.stream(stream):
+                        for ci, call in enumerate(gcalls):
+                            q, k, v = call_inputs(g_in[b][g], call)
+                            launch(ci, call, q, k, v, *g_out[b][g][ci], mask=g_in[b][g].get("block_mask"))
+                    ev_out_ready[b][g].record(stream)
+                ev_in_free[b].record(stream)
+                for g in range(G):
+                    s_out.wait_event(ev_out_ready[b][g])
+                    for (o, l), (ho, hl) in zip(g_out[b][g], host_out):
+                        copy_heads(rt, o, ho, 2, g * hg, hg, False, s_out)
+                        copy_heads(rt, l, hl, 1, g * hg, hg, False, s_out)
+                ev_out_free[b].record(s_out)
 
         pipelined(2)
         torch.cuda.synchronize()
@@ -448,10 +516,17 @@ def run_vdit(args):
         torch.cuda.synchronize()
         barrier()
         e_ms = reduce_max(e0.elapsed_time(e1), dist, dev)
+        # the host results of the last step must equal the device-timed step's
+        # results (same inputs; every head is computed independently)
+        same = all(torch.equal(ho, o.cpu()) and torch.equal(hl, l.cpu()) for (ho, hl), (o, l) in zip(host_out, outs))
+        if not same:
+            raise SystemExit("end-to-end results differ from the device-timed step's")
         e2e = {"value": job_tflops(1, job_step_flops, args.e2e_steps, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps,
-               "overlap": "inputs of step i+1 up and results of step i-1 down while step i computes"}
+               "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps, "head_groups": G,
+               "overlap": (f"heads in {G} groups: group g+1 up and group g-1 down while group g computes; "
+                           "step i+1 up and step i-1 down while step i computes"),
+               "results_checked": "host results of the last step equal the device-timed step's, bit for bit"}
         st, word = vb.vdit_get_device_status(sptr)
         if st != vb.VDIT_OK:
             raise SystemExit(f"device status after the end-to-end steps: {vb.vdit_status_string(st)} ({word:#x})")
@@ -727,6 +802,9 @@ def main():
     ap.add_argument("--impl", choices=("vdit", "reference"), default="vdit")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(wl.WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--e2e-head-groups", type=int, default=8,
+                    help="end-to-end leg: split the heads into this many pipelined copy/compute groups "
+                         "(the largest divisor of H up to it; 1: whole steps)")
     ap.add_argument("--reference-seconds", type=float, default=40.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", choices=("bf16", "fp8"), default="bf16",
