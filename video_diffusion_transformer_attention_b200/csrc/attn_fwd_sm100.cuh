@@ -186,27 +186,59 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 // K = 16 per instruction: 4 steps of 32 bytes inside a half, then the next half.
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc) {
     constexpr uint32_t idesc = make_idesc_bf16(false);
-#pragma unroll
-    for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-        const uint64_t off = (uint64_t(kk >> 2) * kHalfBytes + uint64_t(kk & 3) * 32u) >> 4;
-        umma_ss(d_tmem, q_desc + off, k_desc + off, idesc, kk > 0 ? 1u : 0u);
-    }
+    static_assert(kHalfBytes == 16384, "descriptor offsets below assume 16 KB halves");
+    // The eight K = 16 steps in one asm block: the descriptors advance by
+    // 32 bytes (2 in the >> 4 address field) within a 64-dim half and by
+    // 16 KB (1024) to the second half; the first step overwrites the
+    // accumulator, the others add.  One thread issues these faster as one
+    // block than as eight separate statements.
+    asm volatile(
+        "{\n\t.reg .pred pf, pt;\n\t.reg .b64 a, b;\n\t"
+        "setp.ne.b32 pf, %3, %3;\n\t"
+        "setp.eq.b32 pt, %3, %3;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, pf;\n\t"
+        "add.s64 a, %1, 2;\n\tadd.s64 b, %2, 2;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
+        "add.s64 a, %1, 4;\n\tadd.s64 b, %2, 4;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
+        "add.s64 a, %1, 6;\n\tadd.s64 b, %2, 6;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
+        "add.s64 a, %1, 1024;\n\tadd.s64 b, %2, 1024;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
+        "add.s64 a, %1, 1026;\n\tadd.s64 b, %2, 1026;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
+        "add.s64 a, %1, 1028;\n\tadd.s64 b, %2, 1028;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
+        "add.s64 a, %1, 1030;\n\tadd.s64 b, %2, 1030;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t}" ::"r"(d_tmem),
+        "l"(q_desc), "l"(k_desc), "r"(idesc)
+        : "memory");
 }
 
 // O[128 x 128] (+)= P[128 x keys] * V_tile[keys x 128] for the 64 keys of
 // `half`.  P comes from TMEM (two bf16 per column, 8 columns per K = 16
 // step).  V is the B operand in MN-major form: head dim is contiguous; 64-dim
 // halves are 16 KB apart (leading byte offset), 8-key row groups 1 KB apart
-// (stride byte offset), and each 16-key step advances 16 rows = 2 KB.
+// (stride byte offset), and each 16-key step advances 16 rows = 2 KB.  The
+// four steps are one asm block; the first accumulates unless it starts O.
 __device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, uint64_t v_desc, int half,
                                               bool accumulate) {
     constexpr uint32_t idesc = make_idesc_bf16(true);
-#pragma unroll
-    for (int i = 0; i < kBlockN / 32; ++i) {
-        const int kk = half * (kBlockN / 32) + i;
-        umma_ts(d_tmem, p_tmem + uint32_t(kk) * 8u, v_desc + uint64_t(kk) * (2048u >> 4), idesc,
-                (accumulate || kk > 0) ? 1u : 0u);
-    }
+    const uint32_t a0 = p_tmem + uint32_t(half) * 32u;
+    const uint64_t b0 = v_desc + uint64_t(half) * 512u;
+    asm volatile(
+        "{\n\t.reg .pred p0, pt;\n\t.reg .b32 a;\n\t.reg .b64 b;\n\t"
+        "setp.ne.b32 p0, %4, 0;\n\t"
+        "setp.eq.b32 pt, %3, %3;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n\t"
+        "add.u32 a, %1, 8;\n\tadd.s64 b, %2, 128;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t"
+        "add.u32 a, %1, 16;\n\tadd.s64 b, %2, 256;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t"
+        "add.u32 a, %1, 24;\n\tadd.s64 b, %2, 384;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t}" ::"r"(d_tmem),
+        "r"(a0), "l"(b0), "r"(idesc), "r"((accumulate || half > 0) ? 1u : 0u)
+        : "memory");
 }
 
 // ---------------------------------------------------------------- softmax pieces
