@@ -83,6 +83,31 @@ def test_empty_blocks_and_empty_ctas():
     assert empty[0, 1, 512:768].all() and empty[0, 0, 128:256].all()
 
 
+def test_unequal_key_lists():
+    # The MMA issuer derives each stream entry's owner from the two list
+    # lengths: entries alternate while both lists last, then the longer one's
+    # rest follows.  Cover a long tail on either tile, equal lengths (no
+    # tail), one entry against many, and one empty list.
+    B, H, Sq, Skv = 1, 2, 1024, 1500
+    q, k, v = wl.draw_qkv(B, H, Sq, Skv, 128, seed=54, recipe="rms_qk")
+    nkb = -(-Skv // 128)
+    mask = torch.zeros((B, H, Sq // 128, nkb), dtype=torch.uint8)
+    mask[0, 0, 0, :] = 1          # CTA 0: tile 0 has every key block, tile 1 one
+    mask[0, 0, 1, 5] = 1
+    mask[0, 0, 2, 3] = 1          # CTA 1: tile 0 one block, tile 1 every other block
+    mask[0, 0, 3, ::2] = 1
+    mask[0, 0, 4, 1:9] = 1        # CTA 2: equal lengths, different blocks
+    mask[0, 0, 5, 3:11] = 1
+    mask[0, 0, 6, :4] = 1         # CTA 3: tile 1 has no key block
+    mask[0, 1, 0, 10:] = 1        # head 1: tails of two and ten entries
+    mask[0, 1, 1, :] = 1
+    mask[0, 1, 2, :] = 1
+    mask[0, 1, 3, 7:9] = 1
+    mask[0, 1, 4:8, :] = torch.rand((4, nkb), generator=torch.Generator().manual_seed(55)).lt(0.6).to(torch.uint8)
+    empty = check_all_rows(q, k, v, mask, 1 / math.sqrt(128), "unequal key lists")
+    assert empty[0, 0, 896:1024].all() and not empty[0, 0, :896].any()
+
+
 def test_all_ones_mask_equals_the_full_path_bitwise():
     dev = torch.device("cuda:0")
     B, H, Sq, Skv = 1, 2, 1000, 777
