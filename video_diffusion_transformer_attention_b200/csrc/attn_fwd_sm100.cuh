@@ -71,6 +71,9 @@ constexpr int kControlRegs = 88;    // after setmaxnreg.dec in warpgroup 2
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kNumThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
+constexpr int kStageRows = 32;                             // dense epilogue: one warp's rows, staged in a ring slot
+constexpr int kStageCols = 64;                             // head dims per TMA store box (128 bytes, 128B-swizzled)
+constexpr int kStageWarpBytes = kStageRows * kHeadDim * 2;  // 8 KB per softmax warp: two boxes
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 
 constexpr int kMaskFull = 0;
@@ -278,10 +281,13 @@ __device__ __forceinline__ int sparse_pos(int k, int t, int n0, int n1) {
 // in the dense schedule.  A key block both tiles need appears once for each.
 // The dense, block-causal and cross instantiation keeps the plain issue
 // order, in which both tiles take part in every key tile.
+// tm_o: O as the same 4-D tensor as Q, with 64-dim x 32-row boxes, 128-byte
+// swizzled: the dense epilogue's TMA store unit.
 template <bool kSparse>
 __global__ void __launch_bounds__(kNumThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                          const FwdParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw_base + 1023u) & ~1023u) - raw_base);
@@ -705,6 +711,46 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         if (ok) {
             tc_fence_after_sync();
             const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
+            if constexpr (!kSparse) {
+                // O leaves through shared memory.  Every product that read
+                // ring slot (2 n_kv - 2) mod 4 (the last K tile) completed
+                // before tile 0's last P V, and slot (2 n_kv - 3) mod 4 (the
+                // V tile before the last) before tile 1's, and no load is in
+                // flight any more: tile 0 stages its 128 rows in the first,
+                // tile 1 in the second.  Each thread writes its row (256
+                // bytes) into its warp's 8 KB as two 128B-swizzled 32-row x
+                // 64-dim boxes, and one lane stores both with TMA instead of
+                // 32 rows of 16-byte pieces per store instruction.
+                const int slot = (t == 0 ? 2 * n_kv - 2 : 2 * n_kv - 3) & (kStages - 1);
+                uint8_t* stage = smem + kSmemKV + slot * kTileBytes + quarter * kStageWarpBytes;
+                const uint32_t stage_addr = smem_addr(stage);
+                uint8_t* my_row = stage + lane * 128;
+                const uint32_t swz = uint32_t(lane & 7) << 4;  // 128-byte swizzle: 16-byte chunk ^= row % 8
+#pragma unroll 1
+                for (int c = 0; c < kHeadDim / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + uint32_t(c) * 32u, o);
+                    tmem_ld_wait(o);
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+                    // dims 32c .. 32c+31: box c / 2, 16-byte chunks 4 (c % 2) + i of the row
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        *reinterpret_cast<uint4*>(my_row + (c >> 1) * (kStageWarpBytes / 2) +
+                                                  ((uint32_t((4 * (c & 1) + i) << 4)) ^ swz)) =
+                            make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                const int warp_row0 = q0 + t * kBlockM + quarter * kStageRows;
+                if (lane == 0 && warp_row0 < p.Sq) {
+                    tma_store_4d(&tm_o, stage_addr, 0, h, warp_row0, b);
+                    tma_store_4d(&tm_o, stage_addr + kStageWarpBytes / 2, kStageCols, h, warp_row0, b);
+                    bulk_commit_group();
+                }
+            } else {
             __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.Sq + row) * p.H + h) * kHeadDim;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -727,6 +773,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                         dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
                 }
             }
+            }
             if (p.lse != nullptr && row < p.Sq) {
                 const float m_use = (m == -INFINITY) ? 0.0f : m;
                 p.lse[(static_cast<size_t>(b) * p.H + h) * p.Sq + row] =
@@ -736,6 +783,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     }
 
     // ------------------------------------------------ teardown
+    if (!kSparse && warp < 8 && lane == 0) bulk_wait_all();  // the epilogue's stores are complete
     tc_fence_before_sync();
     __syncthreads();
     if (warp == kMmaWarp) {

@@ -166,6 +166,9 @@ bool encode_bshd(CUtensorMap* map, const void* base, int B, int S, int H) {
 // The output O as a store target for the cross-attention epilogue: the same
 // 4-D view, boxes of 64 head dims x 32 tokens (a warp's rows, 128 bytes each),
 // 128-byte swizzled.  Rows past S are not written.
+static_assert(vdit::kStageCols == vdit::kCrossStageCols && vdit::kStageRows == vdit::kCrossStageRows,
+              "the dense and cross epilogues store O in the same 64-dim x 32-row boxes");
+
 bool encode_bshd_store(CUtensorMap* map, void* base, int B, int S, int H) {
     PFN_cuTensorMapEncodeTiled_v12000 f = encode_fn();
     if (f == nullptr) return false;
@@ -205,12 +208,12 @@ vdit_status launch(const void* q, const void* k, const void* v, void* o, float* 
     p.block_mask = block_mask;
     p.n_qb = (s.Sq + vdit::kSparseBlock - 1) / vdit::kSparseBlock;
     p.n_kvb = (s.Skv + vdit::kSparseBlock - 1) / vdit::kSparseBlock;
+    CUtensorMap to;
+    if (!encode_bshd_store(&to, o, s.B, s.Sq, s.H)) return VDIT_ERR_CUDA;
     if (s.mask_kind == VDIT_MASK_CROSS) {
         // Short key sequence: persistent, two CTAs per SM, one 128-row query tile per item.
         const long long items = static_cast<long long>(p.n_qb) * s.H * s.B;
         const dim3 grid(static_cast<unsigned>(items < ds->cross_grid ? items : ds->cross_grid));
-        CUtensorMap to;
-        if (!encode_bshd_store(&to, o, s.B, s.Sq, s.H)) return VDIT_ERR_CUDA;
         const vdit::CrossSpans rec{cta_spans, max_span_ctas};
         if (!after_norm) {
             vdit::attn_cross_sm100_kernel<<<grid, vdit::kCrossThreads, vdit::kCrossSmemBytes, stream>>>(tq, tk, tv, to,
@@ -235,9 +238,10 @@ vdit_status launch(const void* q, const void* k, const void* v, void* o, float* 
     if (!after_norm) {
         if (s.mask_kind == VDIT_MASK_BLOCK_SPARSE)
             vdit::attn_fwd_sm100_kernel<true><<<grid, vdit::kNumThreads, vdit::kSmemBytesSparse, stream>>>(tq, tk, tv,
-                                                                                                         p);
+                                                                                                         to, p);
         else
-            vdit::attn_fwd_sm100_kernel<false><<<grid, vdit::kNumThreads, vdit::kSmemBytes, stream>>>(tq, tk, tv, p);
+            vdit::attn_fwd_sm100_kernel<false><<<grid, vdit::kNumThreads, vdit::kSmemBytes, stream>>>(tq, tk, tv, to,
+                                                                                                   p);
         return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA;
     }
     // Programmatic dependent of the Q/K norm kernel just queued on this
@@ -253,7 +257,7 @@ vdit_status launch(const void* q, const void* k, const void* v, void* o, float* 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, vdit::attn_fwd_sm100_kernel<false>, tq, tk, tv, p) == cudaSuccess
+    return cudaLaunchKernelEx(&cfg, vdit::attn_fwd_sm100_kernel<false>, tq, tk, tv, to, p) == cudaSuccess
                ? VDIT_OK
                : VDIT_ERR_CUDA;
 }
