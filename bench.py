@@ -440,69 +440,79 @@ def run_vdit(args):
 
     # ---- end to end through the public API, host buffers in and out
     # Every step copies its inputs from pinned host memory and its results
-    # back.  The heads are split into G groups (heads are independent): each
-    # group's Q/K/V go up as one pitched copy per tensor into compact
+    # back.  Across steps, two device buffer sets per kind and three streams
+    # let step i+1's uploads and step i-1's downloads run during step i.  The
+    # first and the last step run in G head groups (heads are independent):
+    # each group's Q/K/V go up as one pitched copy per tensor into compact
     # [B, S, H/G, D] device buffers, the group's calls run as soon as its
     # inputs have landed, and its O/LSE go down while the next group
-    # computes.  Across steps, two device buffer sets and three streams let
-    # step i+1's uploads and step i-1's downloads run during step i.  Only
-    # the first group's upload and the last group's download are exposed.
+    # computes.  Only the first group's upload and the last group's download
+    # are exposed.
     e2e = None
     if args.e2e_steps > 0:
         import dataclasses
         H = w.calls[0].H
         # the largest group count up to the requested one that divides H
         G = max(g for g in range(1, max(1, args.e2e_head_groups) + 1) if H % g == 0)
-        hg = H // G
         rt = cudart()
         host_in = {k: v.pin_memory() for k, v in inp_cpu.items()}
         host_out = [(torch.empty(o.shape, dtype=o.dtype).pin_memory(), torch.empty(l.shape, dtype=l.dtype).pin_memory())
                     for o, l in outs]
         h2d = sum(t.numel() * t.element_size() for t in host_in.values())
         d2h = sum(o.numel() * o.element_size() + l.numel() * l.element_size() for o, l in host_out)
-        gcalls = [dataclasses.replace(c, H=hg) for c in w.calls]
+        class BufferSet:
+            """Device inputs/outputs of one step, split into `ng` head groups."""
 
-        def group_shape(t, axis):
-            return tuple(hg if a == axis else n for a, n in enumerate(t.shape))
+            def __init__(self, ng):
+                self.ng, self.hg = ng, H // ng
+                self.calls = [dataclasses.replace(c, H=self.hg) for c in w.calls]
 
-        # [buffer set][group] -> device tensors
-        g_in = [[{k: torch.empty(group_shape(v, HEAD_AXIS[k]), dtype=v.dtype, device=dev) for k, v in inp.items()}
-                 for _ in range(G)] for _ in range(2)]
-        g_out = [[[(torch.empty(group_shape(o, 2), dtype=o.dtype, device=dev),
-                    torch.empty(group_shape(l, 1), dtype=l.dtype, device=dev)) for o, l in outs]
-                  for _ in range(G)] for _ in range(2)]
+                def shape(t, axis):
+                    return tuple(self.hg if a == axis else n for a, n in enumerate(t.shape))
+
+                self.inp = [{k: torch.empty(shape(v, HEAD_AXIS[k]), dtype=v.dtype, device=dev) for k, v in inp.items()}
+                            for _ in range(ng)]
+                self.out = [[(torch.empty(shape(o, 2), dtype=o.dtype, device=dev),
+                              torch.empty(shape(l, 1), dtype=l.dtype, device=dev)) for o, l in outs] for _ in range(ng)]
+                self.in_ready = [torch.cuda.Event() for _ in range(ng)]
+                self.out_ready = [torch.cuda.Event() for _ in range(ng)]
+                self.in_free, self.out_free = torch.cuda.Event(), torch.cuda.Event()
+                self.used = False
+
+        # Only the first step's uploads and the last step's downloads have no
+        # neighbouring compute to hide behind, so those two steps run in head
+        # groups; the steps between run whole (one launch per call, no
+        # per-group wave tails), their copies overlapping the neighbours'.
+        sets = {(g, b): BufferSet(g) for g in sorted({G, 1}) for b in range(2)}
         s_in = torch.cuda.Stream(device=dev)
         s_out = torch.cuda.Stream(device=dev)
-        ev_in_ready = [[torch.cuda.Event() for _ in range(G)] for _ in range(2)]
-        ev_out_ready = [[torch.cuda.Event() for _ in range(G)] for _ in range(2)]
-        ev_in_free = [torch.cuda.Event() for _ in range(2)]
-        ev_out_free = [torch.cuda.Event() for _ in range(2)]
 
         def pipelined(n_steps):
             for i in range(n_steps):
-                b = i % 2
-                if i >= 2:
-                    s_in.wait_event(ev_in_free[b])
-                for g in range(G):
+                bs = sets[(G if i in (0, n_steps - 1) else 1, i % 2)]
+                if bs.used:
+                    s_in.wait_event(bs.in_free)
+                for g in range(bs.ng):
                     for k_, v_ in host_in.items():
-                        copy_heads(rt, g_in[b][g][k_], v_, HEAD_AXIS[k_], g * hg, hg, True, s_in)
-                    ev_in_ready[b][g].record(s_in)
-                if i >= 2:
-                    stream.wait_event(ev_out_free[b])
-                for g in range(G):
-                    stream.wait_event(ev_in_ready[b][g])
+                        copy_heads(rt, bs.inp[g][k_], v_, HEAD_AXIS[k_], g * bs.hg, bs.hg, True, s_in)
+                    bs.in_ready[g].record(s_in)
+                if bs.used:
+                    stream.wait_event(bs.out_free)
+                for g in range(bs.ng):
+                    stream.wait_event(bs.in_ready[g])
                     with torch.cuda.stream(stream):
-                        for ci, call in enumerate(gcalls):
-                            q, k, v = call_inputs(g_in[b][g], call)
-                            launch(ci, call, q, k, v, *g_out[b][g][ci], mask=g_in[b][g].get("block_mask"))
-                    ev_out_ready[b][g].record(stream)
-                ev_in_free[b].record(stream)
-                for g in range(G):
-                    s_out.wait_event(ev_out_ready[b][g])
-                    for (o, l), (ho, hl) in zip(g_out[b][g], host_out):
-                        copy_heads(rt, o, ho, 2, g * hg, hg, False, s_out)
-                        copy_heads(rt, l, hl, 1, g * hg, hg, False, s_out)
-                ev_out_free[b].record(s_out)
+                        for ci, call in enumerate(bs.calls):
+                            q, k, v = call_inputs(bs.inp[g], call)
+                            launch(ci, call, q, k, v, *bs.out[g][ci], mask=bs.inp[g].get("block_mask"))
+                    bs.out_ready[g].record(stream)
+                bs.in_free.record(stream)
+                for g in range(bs.ng):
+                    s_out.wait_event(bs.out_ready[g])
+                    for (o, l), (ho, hl) in zip(bs.out[g], host_out):
+                        copy_heads(rt, o, ho, 2, g * bs.hg, bs.hg, False, s_out)
+                        copy_heads(rt, l, hl, 1, g * bs.hg, bs.hg, False, s_out)
+                bs.out_free.record(s_out)
+                bs.used = True
 
         pipelined(2)
         torch.cuda.synchronize()
@@ -524,8 +534,8 @@ def run_vdit(args):
         e2e = {"value": job_tflops(1, job_step_flops, args.e2e_steps, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps, "head_groups": G,
-               "overlap": (f"heads in {G} groups: group g+1 up and group g-1 down while group g computes; "
-                           "step i+1 up and step i-1 down while step i computes"),
+               "overlap": (f"first and last step in {G} head groups (group g+1 up / g-1 down while group g "
+                           "computes); step i+1 up and step i-1 down while step i computes"),
                "results_checked": "host results of the last step equal the device-timed step's, bit for bit"}
         st, word = vb.vdit_get_device_status(sptr)
         if st != vb.VDIT_OK:
