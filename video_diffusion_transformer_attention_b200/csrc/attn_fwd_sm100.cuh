@@ -83,7 +83,6 @@ constexpr int kMaskBlockSparse = 3;
 constexpr int kSparseBlock = 128;        // block-mask granularity = the 128-row/128-key tiles
 constexpr int kMaxSparseKvBlocks = 2048; // key blocks a block-sparse call may have (Skv <= 262,144)
 constexpr int kMaxSparseEntries = 2 * kMaxSparseKvBlocks;  // both query tiles' key lists, interleaved
-constexpr uint16_t kListKvMask = 0x3FFF; // list entry: key block | owner query tile << 14
 constexpr int kListWarp = 10;
 
 // Device status word codes (OR-ed together).
@@ -266,19 +265,13 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&s)[32], uint64_t scal
 
 // ---------------------------------------------------------------- kernel
 
-// Position in the block-sparse stream of entry k of query tile t's key list,
-// when tile 0's list has n0 entries and tile 1's n1: the lists alternate
-// (0, 1, 0, 1, ...) while both last, then the longer one's rest follows.
-__device__ __forceinline__ int sparse_pos(int k, int t, int n0, int n1) {
-    const int both = min(n0, n1);
-    return k < both ? 2 * k + t : 2 * both + (k - both);
-}
-
 // kSparse: the block-sparse instantiation.  Each query tile walks only the
-// key blocks its own mask row allows; the two tiles' lists are interleaved
-// into one stream of (key block, owner tile) entries, which the producer
-// loads in order, so the tiles take turns with the tensor core and MUFU as
-// in the dense schedule.  A key block both tiles need appears once for each.
+// key blocks its own mask row allows; the two tiles' lists (n0 and n1
+// entries) are interleaved into one stream, which the producer loads in
+// order: entry k of tile t's list is stream entry 2k + t while k < both =
+// min(n0, n1), then the longer list's rest follows (its entry k at 2 both +
+// k - both).  So the tiles take turns with the tensor core and MUFU as in the
+// dense schedule.  A key block both tiles need appears once for each.
 // The dense, block-causal and cross instantiation keeps the plain issue
 // order, in which both tiles take part in every key tile.
 // tm_o: O as the same 4-D tensor as Q, with 64-dim x 32-row boxes, 128-byte
@@ -328,34 +321,31 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     uint16_t* kv_list = reinterpret_cast<uint16_t*>(smem + kSmemList);
     int* kv_list_len = reinterpret_cast<int*>(smem + kSmemList + kMaxSparseEntries * 2);  // total, n0, n1 (sparse)
     if (kSparse && warp == kListWarp) {
-        // Each query tile's allowed key blocks in ascending order, interleaved
-        // into one stream (sparse_pos), each entry tagged with its owner tile.
+        // Each query tile's allowed key blocks in ascending order, in one
+        // pass: tile 0's list at kv_list[0 ..), tile 1's at
+        // kv_list[kMaxSparseKvBlocks ..).  The stream the producer loads
+        // interleaves them; it is never stored.
         const int qb0 = q0 / kSparseBlock;
         const uint8_t* row0 = p.block_mask + ((static_cast<size_t>(b) * p.H + h) * p.n_qb + qb0) * p.n_kvb;
         const bool has_row1 = qb0 + 1 < p.n_qb;
         const uint32_t below = (1u << lane) - 1u;
-        int n0 = 0, n1 = 0;
-        for (int base = 0; base < p.n_kvb; base += 32) {
-            const int kv = base + lane;
-            n0 += __popc(__ballot_sync(0xffffffffu, kv < p.n_kvb && row0[kv] != 0));
-            n1 += __popc(__ballot_sync(0xffffffffu, has_row1 && kv < p.n_kvb && row0[p.n_kvb + kv] != 0));
-        }
         int c0 = 0, c1 = 0;
+#pragma unroll 4
         for (int base = 0; base < p.n_kvb; base += 32) {
             const int kv = base + lane;
             const bool a0 = kv < p.n_kvb && row0[kv] != 0;
             const bool a1 = has_row1 && kv < p.n_kvb && row0[p.n_kvb + kv] != 0;
             const uint32_t b0 = __ballot_sync(0xffffffffu, a0);
             const uint32_t b1 = __ballot_sync(0xffffffffu, a1);
-            if (a0) kv_list[sparse_pos(c0 + __popc(b0 & below), 0, n0, n1)] = uint16_t(kv);
-            if (a1) kv_list[sparse_pos(c1 + __popc(b1 & below), 1, n0, n1)] = uint16_t(kv | (1 << 14));
+            if (a0) kv_list[c0 + __popc(b0 & below)] = uint16_t(kv);
+            if (a1) kv_list[kMaxSparseKvBlocks + c1 + __popc(b1 & below)] = uint16_t(kv);
             c0 += __popc(b0);
             c1 += __popc(b1);
         }
         if (lane == 0) {
-            kv_list_len[0] = n0 + n1;
-            kv_list_len[1] = n0;
-            kv_list_len[2] = n1;
+            kv_list_len[0] = c0 + c1;
+            kv_list_len[1] = c0;
+            kv_list_len[2] = c1;
         }
     }
     tc_fence_before_sync();
@@ -397,7 +387,14 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     break;
                 const uint32_t full = smem_addr(&bars->kv_full[slot]);
                 const CUtensorMap* map = (u & 1) ? &tm_v : &tm_k;
-                const int row = (sparse ? int(kv_list[u >> 1] & kListKvMask) : (u >> 1)) * kBlockN;
+                int blk = u >> 1;
+                if constexpr (kSparse) {  // stream entry u >> 1 -> (tile, list entry)
+                    const int e = u >> 1, n0 = kv_list_len[1], n1 = kv_list_len[2];
+                    const int both2 = 2 * min(n0, n1);
+                    blk = e < both2 ? int(kv_list[(e & 1) * kMaxSparseKvBlocks + (e >> 1)])
+                                    : int(kv_list[(n0 >= n1 ? 0 : kMaxSparseKvBlocks) + (e - both2 / 2)]);
+                }
+                const int row = blk * kBlockN;
                 mbar_arrive_expect_tx(full, kTileBytes);
                 tma_load_4d(sKV + slot * kTileBytes, map, full, 0, h, row, b);
                 tma_load_4d(sKV + slot * kTileBytes + kHalfBytes, map, full, 64, h, row, b);
@@ -466,8 +463,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             // that tile's P V on e comes its S on its next entry (two entries
             // on while both lists last, then the next one), so the two tiles
             // keep taking turns.  Barrier phases count each tile's own entries.
-            // The stream's shape follows from the two list lengths alone
-            // (sparse_pos): entries [0, both2) alternate between the tiles,
+            // The stream's shape follows from the two list lengths alone:
+            // entries [0, both2) alternate between the tiles,
             // the rest belong to the tile with the longer list.  Owner and
             // next entry are register arithmetic, no shared-memory reads.
             const int n0 = kv_list_len[1], n1 = kv_list_len[2];
@@ -576,8 +573,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             // keys of this tile allowed for the row: [0, lim) of the tile
             int lim;
             if (sparse) {
-                const int e = sparse_pos(j, t, kv_list_len[1], kv_list_len[2]);
-                lim = p.Skv - int(kv_list[e] & kListKvMask) * kBlockN;
+                lim = p.Skv - int(kv_list[t * kMaxSparseKvBlocks + j]) * kBlockN;
             } else {
                 lim = kv_lim - j * kBlockN;
             }
