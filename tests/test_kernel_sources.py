@@ -15,7 +15,7 @@ import pytest
 
 CSRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
                     "video_diffusion_transformer_attention_b200", "csrc")
-KERNELS = ["attn_fwd_sm100.cuh", "attn_cross_sm100.cuh", "attn_fwd_fp8_sm100.cuh", "fp8_quant.cuh",
+KERNELS = ["attn_fwd_sm100.cuh", "attn_cross_sm100.cuh", "attn_cross_fp8_sm100.cuh", "attn_fwd_fp8_sm100.cuh", "fp8_quant.cuh",
            "qk_norm.cuh", "attn_merge.cuh", "vsmooth_group.cuh"]
 PTX_HELPERS = ["sm100_ptx.cuh", "sm100_fp8_ptx.cuh"]
 WARP_INTRINSICS = {"__syncwarp", "__any_sync", "__all_sync", "__ballot_sync", "__shfl_sync",

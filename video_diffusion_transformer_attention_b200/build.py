@@ -20,7 +20,7 @@ LIB = os.path.join(HERE, "libvdit_attn.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("vdit_attn.cu", "attn_fwd_sm100.cuh", "sm100_ptx.cuh",
                                            "attn_merge.cuh", "qk_norm.cuh", "fp8_quant.cuh",
                                            "attn_fwd_fp8_sm100.cuh", "sm100_fp8_ptx.cuh", "vsmooth_group.cuh",
-                                           "attn_cross_sm100.cuh")]
+                                           "attn_cross_sm100.cuh", "attn_cross_fp8_sm100.cuh")]
 HEADERS = [os.path.join(INCLUDE, "vdit_attn.h"), os.path.join(INCLUDE, "vdit_attn_testing.h")]
 
 NVCC_FLAGS = [

@@ -16,6 +16,7 @@
 #include "vdit_attn_testing.h"
 #include "attn_fwd_sm100.cuh"
 #include "attn_cross_sm100.cuh"
+#include "attn_cross_fp8_sm100.cuh"
 #include "attn_merge.cuh"
 #include "qk_norm.cuh"
 #include "fp8_quant.cuh"
@@ -94,7 +95,11 @@ void init_device(int dev, DeviceState* st) {
         cudaFuncSetAttribute(vdit::attn_cross_sm100_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
         cudaFuncSetAttribute(vdit::attn_fwd_fp8_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             vdit::kF8SmemBytes) != cudaSuccess) {
+                             vdit::kF8SmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(vdit::attn_cross_fp8_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             vdit::kF8CrossSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(vdit::attn_cross_fp8_sm100_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess) {
         st->status = VDIT_ERR_CUDA;
         return;
     }
@@ -499,15 +504,29 @@ vdit_status fp8_attention_impl(void* o, float* lse, const Shape& s, float scale,
     p.lse = lse;
     p.timeout_ns = kDefaultWaitTimeoutNs;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(grid_x(s.Sq), s.H, s.B);
-    cfg.blockDim = dim3(vdit::kNumThreads);
-    cfg.dynamicSmemBytes = vdit::kF8SmemBytes;
-    cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = after_quantize ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    cfg.stream = stream;
+    if (s.mask_kind == VDIT_MASK_CROSS) {
+        // Short key sequence: persistent, two CTAs per SM, one 128-row query tile per item.
+        const DeviceState* ds = nullptr;
+        if (ensure_device(&dev, &ds) != VDIT_OK) return VDIT_ERR_CUDA;
+        CUtensorMap to;
+        if (!encode_bshd_store(&to, o, s.B, s.Sq, s.H)) return VDIT_ERR_CUDA;
+        const long long items = static_cast<long long>(nqb) * s.H * s.B;
+        cfg.gridDim = dim3(static_cast<unsigned>(items < ds->cross_grid ? items : ds->cross_grid));
+        cfg.blockDim = dim3(vdit::kCrossThreads);
+        cfg.dynamicSmemBytes = vdit::kF8CrossSmemBytes;
+        return cudaLaunchKernelEx(&cfg, vdit::attn_cross_fp8_sm100_kernel, tq, tk, tvt, to, p) == cudaSuccess
+                   ? VDIT_OK
+                   : VDIT_ERR_CUDA;
+    }
+    cfg.gridDim = dim3(grid_x(s.Sq), s.H, s.B);
+    cfg.blockDim = dim3(vdit::kNumThreads);
+    cfg.dynamicSmemBytes = vdit::kF8SmemBytes;
     return cudaLaunchKernelEx(&cfg, vdit::attn_fwd_fp8_sm100_kernel, tq, tk, tvt, p) == cudaSuccess ? VDIT_OK
                                                                                                   : VDIT_ERR_CUDA;
 }
