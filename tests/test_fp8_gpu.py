@@ -199,3 +199,40 @@ def test_fp8_attention_sampled_rows_at_a_wan_shape():
     groups = [np.nonzero(rows[:, 1] == h)[0] for h in range(call.H)]
     res = check_expcast_parity(og, o_p, lg, l_p, s_o, s_l, groups, f"fp8 plain {name} sampled")
     assert res["ok"], res
+
+
+def test_fp8_cross_attention_sampled_rows_at_the_bench_shape():
+    # Sq = 75,600, H = 40, Skv = 512 text tokens: the persistent cross kernel
+    # takes ~80 query tiles per CTA, so its barrier phases run across items
+    name = "wan21_14b_720p"
+    call = wl.WORKLOADS[name].calls[1]
+    inp = wl.workload_inputs(name)
+    q, k, v = inp["q"], inp["k_text"], inp["v_text"]
+    o, lse = _run_fp8(q, k, v, call.mask_kind, call.chunk_tokens, call.scale)
+    rows = wl.sample_rows(call.B, call.H, call.Sq, 8, seed=97)
+    quant = (f8.quantize_qk(wl.bf16_bits(q)), f8.quantize_qk(wl.bf16_bits(k)), f8.vsmooth(wl.bf16_bits(v)))
+    o_r, l_r = f8.attention_fp8(None, None, None, call.scale, call.mask_kind, call.chunk_tokens, rows=rows,
+                                quantized=quant)
+    og = np.stack([o[b, i, h] for b, h, i in rows])
+    lg = np.array([lse[b, h, i] for b, h, i in rows])
+    res = check_parity(og, o_r, lg, l_r, None, f"fp8 {name} cross sampled", excess_bar=None)
+    assert res["ok"], res
+    o_p, l_p, s_o, s_l = f8.attention_fp8_plain(None, None, None, call.scale, call.mask_kind, call.chunk_tokens,
+                                                 rows=rows, quantized=quant, spread=True)
+    groups = [np.nonzero(rows[:, 1] == h)[0] for h in range(call.H)]
+    res = check_expcast_parity(og, o_p, lg, l_p, s_o, s_l, groups, f"fp8 plain {name} cross sampled")
+    assert res["ok"], res
+
+
+def test_fp8_cross_attention_all_rows_several_items_per_cta():
+    # 600 query tiles over 296 CTAs: every CTA runs two or three items
+    B, H, Sq, Skv = 1, 4, 128 * 150 - 37, 300
+    q, k, v = wl.draw_qkv(B, H, Sq, Skv, 128, seed=98, recipe="rms_qk")
+    scale = 1 / math.sqrt(128)
+    o, lse = _run_fp8(q, k, v, vb.VDIT_MASK_CROSS, 0, scale)
+    o_r, l_r = f8.attention_fp8(wl.bf16_bits(q), wl.bf16_bits(k), wl.bf16_bits(v), scale, vb.VDIT_MASK_CROSS, 0)
+    og, lg = _flat(o, lse, B, H)
+    orr, lr = _flat(o_r, l_r, B, H)
+    res = check_parity(og, orr, lg, lr, [np.arange(i * Sq, (i + 1) * Sq) for i in range(B * H)],
+                       "fp8 cross, several items per CTA", excess_bar=None)
+    assert res["ok"], res
