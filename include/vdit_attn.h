@@ -253,7 +253,9 @@ vdit_status vdit_attn_fwd_qknorm_noalloc(const void* q, const void* k,
  *    than 24 codes.
  * O is bf16 and LSE fp32 as in vdit_attn_fwd; the result differs from
  * vdit_attn_fwd by the 8-bit quantisation (a few percent relative RMS on
- * iid data).  Masks: FULL, BLOCK_CAUSAL, CROSS.  D must be 128.
+ * iid data).  Masks: FULL, BLOCK_CAUSAL, CROSS; as in vdit_attn_fwd, CROSS
+ * takes the short-key schedule (persistent CTAs, two per SM, one 128-row
+ * query tile at a time) with the same per-row arithmetic.  D must be 128.
  *
  * The caller owns a device workspace (256-byte aligned, size from
  * vdit_attn_fp8_plan) that holds the codes; its parts, in this order, are
