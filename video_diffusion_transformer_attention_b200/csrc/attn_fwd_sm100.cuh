@@ -276,7 +276,7 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&s)[32], uint64_t scal
 // order, in which both tiles take part in every key tile.
 // tm_o: O as the same 4-D tensor as Q, with 64-dim x 32-row boxes, 128-byte
 // swizzled: the dense epilogue's TMA store unit.
-template <bool kSparse>
+template <bool kSparse, bool kLongFirst = false>
 __global__ void __launch_bounds__(kNumThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -291,7 +291,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const int lane = int(threadIdx.x & 31);
     const int h = int(blockIdx.y);
     const int b = int(blockIdx.z);
-    const int q0 = int(blockIdx.x) * (kQTiles * kBlockM);
+    // kLongFirst (block-causal): the CTAs of later chunks walk more key tiles;
+    // dispatching them first (blocks start in blockIdx order) leaves short
+    // CTAs, not long ones, to fill the end of the grid.
+    const int q_pair = kLongFirst ? int(gridDim.x - 1u - blockIdx.x) : int(blockIdx.x);
+    const int q0 = q_pair * (kQTiles * kBlockM);
 
     if (threadIdx.x == 0) {
         for (int t = 0; t < kQTiles; ++t) {

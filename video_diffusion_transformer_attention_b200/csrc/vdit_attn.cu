@@ -89,6 +89,8 @@ void init_device(int dev, DeviceState* st) {
                              vdit::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(vdit::attn_fwd_sm100_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              vdit::kSmemBytesSparse) != cudaSuccess ||
+        cudaFuncSetAttribute(vdit::attn_fwd_sm100_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             vdit::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(vdit::attn_cross_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              vdit::kCrossSmemBytes) != cudaSuccess ||
         // all of the unified L1 / shared storage as shared memory: two CTAs fit
@@ -244,6 +246,9 @@ vdit_status launch(const void* q, const void* k, const void* v, void* o, float* 
         if (s.mask_kind == VDIT_MASK_BLOCK_SPARSE)
             vdit::attn_fwd_sm100_kernel<true><<<grid, vdit::kNumThreads, vdit::kSmemBytesSparse, stream>>>(tq, tk, tv,
                                                                                                          to, p);
+        else if (s.mask_kind == VDIT_MASK_BLOCK_CAUSAL)
+            vdit::attn_fwd_sm100_kernel<false, true><<<grid, vdit::kNumThreads, vdit::kSmemBytes, stream>>>(tq, tk, tv,
+                                                                                                         to, p);
         else
             vdit::attn_fwd_sm100_kernel<false><<<grid, vdit::kNumThreads, vdit::kSmemBytes, stream>>>(tq, tk, tv, to,
                                                                                                    p);
@@ -262,6 +267,10 @@ vdit_status launch(const void* q, const void* k, const void* v, void* o, float* 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (s.mask_kind == VDIT_MASK_BLOCK_CAUSAL)
+        return cudaLaunchKernelEx(&cfg, vdit::attn_fwd_sm100_kernel<false, true>, tq, tk, tv, to, p) == cudaSuccess
+                   ? VDIT_OK
+                   : VDIT_ERR_CUDA;
     return cudaLaunchKernelEx(&cfg, vdit::attn_fwd_sm100_kernel<false>, tq, tk, tv, to, p) == cudaSuccess
                ? VDIT_OK
                : VDIT_ERR_CUDA;
