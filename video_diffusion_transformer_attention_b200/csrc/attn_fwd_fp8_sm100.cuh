@@ -298,6 +298,10 @@ __device__ __forceinline__ void fp8_softmax_rows(const Fp8FwdParams& p, Fp8Barri
     }
 }
 
+// kLongFirst (block-causal): block x takes query-tile pair gridDim.x - 1 - x,
+// so each head's CTAs with the most key tiles start first, as in the bf16
+// kernel.
+template <bool kLongFirst = false>
 __global__ void __launch_bounds__(kNumThreads, 1)
     attn_fwd_fp8_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_vt, const Fp8FwdParams p) {
@@ -311,7 +315,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const int lane = int(threadIdx.x & 31);
     const int h = int(blockIdx.y);
     const int b = int(blockIdx.z);
-    const int q0 = int(blockIdx.x) * (kQTiles * kBlockM);
+    const int q0 = (kLongFirst ? int(gridDim.x - 1u - blockIdx.x) : int(blockIdx.x)) * (kQTiles * kBlockM);
     const size_t bh = static_cast<size_t>(b) * p.H + h;
 
     if (threadIdx.x == 0) {

@@ -96,7 +96,9 @@ void init_device(int dev, DeviceState* st) {
         // all of the unified L1 / shared storage as shared memory: two CTAs fit
         cudaFuncSetAttribute(vdit::attn_cross_sm100_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
-        cudaFuncSetAttribute(vdit::attn_fwd_fp8_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(vdit::attn_fwd_fp8_sm100_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             vdit::kF8SmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(vdit::attn_fwd_fp8_sm100_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              vdit::kF8SmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(vdit::attn_cross_fp8_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              vdit::kF8CrossSmemBytes) != cudaSuccess ||
@@ -536,8 +538,13 @@ vdit_status fp8_attention_impl(void* o, float* lse, const Shape& s, float scale,
     cfg.gridDim = dim3(grid_x(s.Sq), s.H, s.B);
     cfg.blockDim = dim3(vdit::kNumThreads);
     cfg.dynamicSmemBytes = vdit::kF8SmemBytes;
-    return cudaLaunchKernelEx(&cfg, vdit::attn_fwd_fp8_sm100_kernel, tq, tk, tvt, p) == cudaSuccess ? VDIT_OK
-                                                                                                  : VDIT_ERR_CUDA;
+    if (s.mask_kind == VDIT_MASK_BLOCK_CAUSAL)
+        return cudaLaunchKernelEx(&cfg, vdit::attn_fwd_fp8_sm100_kernel<true>, tq, tk, tvt, p) == cudaSuccess
+                   ? VDIT_OK
+                   : VDIT_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, vdit::attn_fwd_fp8_sm100_kernel<false>, tq, tk, tvt, p) == cudaSuccess
+               ? VDIT_OK
+               : VDIT_ERR_CUDA;
 }
 
 // ------------------------------------------------------------ LSE merge
