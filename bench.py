@@ -582,7 +582,8 @@ def run_vdit(args):
             # is reported beside it.
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_burst, "unit": "TFLOP/s",
                          "frac": achieved / peak_burst,
-                         "traffic": recorded_traffic() if args.workload == WORKLOAD and args.path == "bf16" else None,
+                         "traffic": (recorded_traffic() if args.workload == WORKLOAD and args.path == "bf16" and not args.heads
+                                     and heads is None else None),
                          "kernel": ("attn_fwd_fp8_sm100_kernel (self-attention launch)" if args.path == "fp8" else
                                     "attn_fwd_sm100_kernel (self-attention launch)" if not args.qknorm else
                                     "qk_rms_norm_kernel + attn_fwd_sm100_kernel (self-attention call)"),
