@@ -55,11 +55,22 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def _code_lines(text):
+    """The source's code without // comments and blank lines: a comment edit
+    does not change the kernel the traffic record was taken on."""
+    out = []
+    for line in text.splitlines():
+        code = line.split("//", 1)[0].rstrip()
+        if code:
+            out.append(code)
+    return "\n".join(out)
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     for f in ("attn_fwd_sm100.cuh", "sm100_ptx.cuh"):
-        with open(os.path.join(ROOT, "video_diffusion_transformer_attention_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "video_diffusion_transformer_attention_b200", "csrc", f)) as fh:
+            h.update(_code_lines(fh.read()).encode())
     return h.hexdigest()
 
 

@@ -27,14 +27,18 @@
 //     current reference first, and one of them exceeds it by more than the
 //     threshold only if their exponentials sum to more than 2^8; keys 64-127
 //     are checked by their max.  The exact tile max is taken only when a
-//     check fires.
+//     check fires;
+//   * O leaves through shared memory: after its last P V each tile stages
+//     its rows in a ring slot that no product or load uses any more, and one
+//     lane per warp stores them with TMA.
 //
 // Roles (384 threads, three warpgroups):
 //   warps 0-3   softmax + correction + epilogue of query tile 0
 //   warps 4-7   softmax + correction + epilogue of query tile 1
 //   warp  8     TMA producer (Q once, then K_j, V_j into a 4-slot ring)
 //   warp  9     TMEM allocator and single-thread tcgen05.mma issuer
-//   warps 10-11 idle
+//   warp  10    block-sparse only: builds the two tiles' key lists, then idles
+//   warp  11    idle
 // The kernel is launched at 168 registers a thread (384 x 168 = 64,512); the
 // softmax warpgroups then raise theirs to 208 and the third lowers its to 88
 // (2 x 128 x 208 + 128 x 88 = 64,512, the same total).
